@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Throughput of speculative-sampling verification on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step = one ``spec_verify`` call over one batch of the synthetic
+quantized-self-draft workload (B=64 requests, k=8 drafts, V=151,936, bf16
+logits, T=1) with its inputs already resident in HBM: the row-statistics
+kernel over every used row, then the acceptance scan and the final draw.
+Rank 0 prints one JSON line.
+
+* value        verified draft positions/s over all ranks (sum of draft
+               lengths per call x calls / max-over-ranks device time)
+* e2e          the same metric through the host entry point
+               (spec_verify_host): pinned host inputs copied in, results
+               copied out, every step
+* roofline     the row-statistics kernel: algorithmic bytes (every logit of
+               every used row, read once) / its CUDA-event time, against the
+               measured HBM copy bandwidth
+* cpu_baseline the CPU oracle on the host cores (single thread), on a bounded
+               sample of the same workload
+
+With N > 1 (torchrun), every rank verifies its own batch (weak scaling); no
+collective touches the data path, only the timing barrier and the max over
+ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from speculative_decoding_verification_92_b200.workload import CONFIGS, config_seed, make_workload  # noqa: E402
+
+METRIC = "verified draft positions/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "positions/s"
+FALLBACK_HBM_GBS = 6650.0
+MAX_REQUESTS_PER_STATS_LAUNCH = 4096     # mirrors the library's launch split
+MAX_REQUESTS_PER_DRAW_LAUNCH = 65535
+TRAFFIC_FILE = ROOT / "profiles" / "row_stats_traffic.json"
+
+NVML_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--stats-kernel", default="auto", choices=["auto", "tma", "vec16", "scalar"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--greedy", action="store_true", help="time the greedy (prefix-match) form instead")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# workload bookkeeping
+
+
+def make_rank_workload(cfg: int, rank: int):
+    params = dict(CONFIGS[cfg])
+    return make_workload(seed=config_seed(cfg) + 7919 * rank, **params)
+
+
+def stats_pass_bytes(w, greedy=False) -> int:
+    """Algorithmic bytes of one call: every logit of every row the rule must
+    read (target rows 0..L_b, draft rows 0..L_b-1), once."""
+    L = w.draft_lens.astype(np.int64)
+    rows = int((L + 1).sum())
+    if w.draft is not None and not greedy:
+        rows += int(L.sum())
+    return rows * w.V * w.esize
+
+
+def input_bytes(w, greedy=False) -> int:
+    n = w.target.nbytes + w.tokens.nbytes
+    if w.draft is not None and not greedy:
+        n += w.draft.nbytes
+    if w.lens is not None:
+        n += w.lens.nbytes
+    if not greedy:
+        n += w.uniforms.nbytes
+    return int(n)
+
+
+def workload_desc(w, cfg) -> dict:
+    return {
+        "workload": f"{w.name}: B={w.B} k={w.k_max} V={w.V} {w.dtype} T={w.temperature}"
+                    + (" one-hot q (no draft logits)" if w.draft is None else " draft logits")
+                    + (" L in {0,4,12}" if w.lens is not None else ""),
+        "config_id": cfg, "B": w.B, "k_max": w.k_max, "V": w.V, "input_dtype": w.dtype,
+        "temperature": w.temperature, "draft": "ids" if w.draft is None else "logits",
+        "positions_per_step": w.positions, "seed": config_seed(cfg),
+    }
+
+
+def measured_peak():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            d = json.loads(p.read_text())
+            return float(d["hbm_gbs"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(kernel_variant: str, cfg: int):
+    """Per-launch DRAM bytes of the row-statistics kernel from the committed
+    ncu summary, only if it was taken on the current kernel sources."""
+    if not TRAFFIC_FILE.exists():
+        return None
+    try:
+        from speculative_decoding_verification_92_b200 import build as _b
+        d = json.loads(TRAFFIC_FILE.read_text())
+        if d.get("source_hash") != _b.source_hash():
+            return None
+        e = d.get("per_config", {}).get(str(cfg), {}).get(kernel_variant)
+        return None if e is None else float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report what we have
+            log(f"clock sampling unavailable: {e}")
+        self.period = period_s
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                try:
+                    r = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    r = n.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.reasons |= int(r)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.ok:
+            self.thread.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [v for k, v in NVML_REASONS.items() if self.reasons & k]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing
+
+
+def time_oracle(w, n_requests: int, seconds: float, greedy=False, min_reps=1):
+    """Run the oracle on the first n_requests of the batch until `seconds`
+    have passed (at least min_reps times); returns (positions/s, reps,
+    positions per rep, seconds)."""
+    from oracle import default
+    orc = default()
+    sl = slice(0, n_requests)
+    lens = None if w.lens is None else w.lens[sl]
+    u = w.uniforms[sl].astype(np.float64)
+    positions = int(w.draft_lens[sl].sum())
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        orc.verify(w.target[sl], None if (greedy or w.draft is None) else w.draft[sl], w.tokens[sl], lens,
+                   None if greedy else u, w.temperature, greedy, V=w.V)
+        reps += 1
+        el = time.perf_counter() - t0
+        if reps >= min_reps and el >= seconds:
+            break
+    return positions * reps / el, reps, positions, el
+
+
+# ---------------------------------------------------------------------------
+
+
+def run_reference(args):
+    """CPU oracle arm: rank 0 alone; every step verifies a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = make_rank_workload(args.config, 0)
+    from oracle import default
+    orc = default()
+    # calibrate the per-request cost, then size the per-step sample so that
+    # warm-up + steps stay within about two minutes
+    t0 = time.perf_counter()
+    orc.verify(w.target[:1], None if w.draft is None else w.draft[:1], w.tokens[:1],
+               None if w.lens is None else w.lens[:1], w.uniforms[:1].astype(np.float64), w.temperature,
+               args.greedy, V=w.V)
+    per_req = max(time.perf_counter() - t0, 1e-4)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n_req = int(max(1, min(w.B, budget // per_req)))
+    sl = slice(0, n_req)
+    lens = None if w.lens is None else w.lens[sl]
+    u = w.uniforms[sl].astype(np.float64)
+    draft = None if (w.draft is None or args.greedy) else w.draft[sl]
+    positions = int(w.draft_lens[sl].sum())
+    for _ in range(args.warmup):
+        orc.verify(w.target[sl], draft, w.tokens[sl], lens, u, w.temperature, args.greedy, V=w.V)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        orc.verify(w.target[sl], draft, w.tokens[sl], lens, u, w.temperature, args.greedy, V=w.V)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = positions * args.steps / total
+    sample = f"first {n_req} of {w.B} requests ({positions} draft positions) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_desc(w, args.config),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours_impl(args)
+
+
+def run_ours_impl(args):
+    import torch
+    import torch.distributed as dist
+
+    import speculative_decoding_verification_92_b200 as sv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        log(f"--gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
+    n = world
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if n > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if n > 1:
+            dist.barrier()
+
+    sv.library()  # build / load before timing anything
+    w = make_rank_workload(args.config, rank)
+    greedy = bool(args.greedy)
+    kernel = {"auto": sv.StatsKernel.AUTO, "tma": sv.StatsKernel.TMA, "vec16": sv.StatsKernel.VEC16,
+              "scalar": sv.StatsKernel.SCALAR}[args.stats_kernel]
+
+    def dev_tensor(a, bf16=False):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if bf16:
+            t = t.view(torch.bfloat16)
+        return t.to(dev)
+
+    is_bf16 = w.dtype == "bf16"
+    target = dev_tensor(w.target, is_bf16)
+    draft = None if (w.draft is None or greedy) else dev_tensor(w.draft, is_bf16)
+    tokens = dev_tensor(w.tokens)
+    lens = None if w.lens is None else dev_tensor(w.lens)
+    uniforms = None if greedy else dev_tensor(w.uniforms)
+    out = (torch.empty(w.B, dtype=torch.int32, device=dev),
+           torch.empty(w.B, w.k_max + 1, dtype=torch.int32, device=dev))
+    ws = torch.empty(max(sv.workspace_bytes(w.B, w.k_max, w.V, sv.BF16 if is_bf16 else sv.F32), 256),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    in_bytes = input_bytes(w, greedy)
+    flush_buf = None
+    if in_bytes < 2 * l2:
+        flush_buf = torch.empty(4 * l2 // 4, dtype=torch.int32, device=dev)
+    l2_note = (f"inputs {in_bytes / 1e6:.1f} MB > 2 x L2 ({l2 / 2**20:.0f} MiB): no flush" if flush_buf is None
+               else f"inputs {in_bytes / 1e6:.1f} MB < 2 x L2: L2 flushed (write {flush_buf.numel() * 4 / 2**20:.0f}"
+                    f" MiB) before every step, outside each step's events")
+
+    def step(events=None):
+        sv.spec_verify(target, draft, tokens, lens, uniforms, w.temperature, greedy, V=w.V, out=out,
+                       workspace=ws, stream=stream, stats_kernel=kernel, events=events)
+
+    def new_event():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    step_ev = [(new_event(), new_event()) for _ in range(K)]
+    k1_ev = [(new_event(), new_event()) for _ in range(K)]
+    g0, g1 = new_event(), new_event()
+    torch.cuda.synchronize()
+
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        g0.record(stream)
+        for i in range(K):
+            if flush_buf is not None:
+                flush_buf.fill_(i)
+            step_ev[i][0].record(stream)
+            step(events=k1_ev[i])
+            step_ev[i][1].record(stream)
+        g1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    k1_ms = [a.elapsed_time(b) for a, b in k1_ev]
+    region_ms = g0.elapsed_time(g1)
+    t_rank = sum(step_ms) if flush_buf is not None else region_ms
+    t_max = t_rank
+    if n > 1:
+        t = torch.tensor([t_rank], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    positions = w.positions
+    value = n * positions * K / (t_max / 1e3)
+    ms_per_step = t_max / K
+
+    # parity spot check of the timed outputs (host side, cheap): accept lengths in range
+    g_len = out[0].cpu().numpy()
+    assert np.all((g_len >= 0) & (g_len <= w.draft_lens)), "timed run produced invalid outputs"
+    accept_rate = float(g_len.sum() / max(1, positions))
+
+    # ---------------- end to end through the host entry point ----------------
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = lambda a, bf=False: (torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16) if bf
+                                   else torch.from_numpy(np.ascontiguousarray(a))).pin_memory()
+        h_target = pin(w.target, is_bf16)
+        h_draft = None if draft is None else pin(w.draft, is_bf16)
+        h_tokens, h_lens = pin(w.tokens), (None if w.lens is None else pin(w.lens))
+        h_u = None if greedy else pin(w.uniforms)
+        h_out = (torch.empty(w.B, dtype=torch.int32).pin_memory(),
+                 torch.empty(w.B, w.k_max + 1, dtype=torch.int32).pin_memory())
+        staging = torch.empty(sv.host_staging_bytes(w.B, w.k_max, w.V, sv.BF16 if is_bf16 else sv.F32,
+                                                    has_draft=h_draft is not None, has_lens=h_lens is not None),
+                              dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            sv.spec_verify_host(h_target, h_draft, h_tokens, h_lens, h_u, w.temperature, greedy, V=w.V,
+                                out=h_out, staging=staging, workspace=ws, stream=stream)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ev = [(new_event(), new_event()) for _ in range(args.e2e_steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(args.e2e_steps):
+            ev[i][0].record(stream)
+            e2e_step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in ev)
+        if n > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        assert np.array_equal(h_out[0].numpy(), g_len), "host entry point disagrees with device entry point"
+        e2e = {"value": n * positions * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": int(h_out[0].nbytes + h_out[1].nbytes),
+               "steps": args.e2e_steps, "ms_per_step": e2e_ms / args.e2e_steps}
+
+    # ---------------- roofline of the row-statistics kernel ----------------
+    peak, peak_kind = measured_peak()
+    alg = stats_pass_bytes(w, greedy)
+    k1_mean = statistics.fmean(k1_ms)
+    achieved = alg / (k1_mean / 1e3) / 1e9
+    variant = "tma" if args.stats_kernel == "auto" else args.stats_kernel
+    traffic = committed_traffic(variant, args.config)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic, "peak_kind": f"{peak_kind} (copy bandwidth, MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6650 GB/s",
+                "kernel": f"row_stats ({variant})", "algorithmic_bytes_per_launch": alg,
+                "kernel_ms": k1_mean, "kernel_ms_p10": float(np.percentile(k1_ms, 10)),
+                "whole_step_gbs": alg / (ms_per_step / 1e3) / 1e9}
+
+    launches_per_call = math.ceil(w.B / MAX_REQUESTS_PER_STATS_LAUNCH) + math.ceil(w.B / MAX_REQUESTS_PER_DRAW_LAUNCH)
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
+    cpu = None
+    if rank == 0 and n == 1 and not args.no_cpu_baseline:
+        v, reps, pos, el = time_oracle(w, w.B, args.cpu_seconds, greedy)
+        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"whole batch ({w.B} requests, {pos} draft positions) x {reps} passes, {el:.1f} s,"
+                         f" single-threaded C, fp64"}
+
+    if rank == 0:
+        cfgd = workload_desc(w, args.config)
+        cfgd.update({"parallelism": f"replicas{n}" if n > 1 else "single",
+                     "sharding": "each rank verifies its own batch; no data-path collective",
+                     "l2": l2_note, "stats_kernel": variant, "greedy": greedy})
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": K, "warmup": W,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic", "config": cfgd,
+            "e2e": e2e, "gpu_launches": K * launches_per_call, "roofline": roofline,
+            "cpu_baseline": cpu, "clocks": clocks.summary(),
+            "hbm_gbs": alg / (ms_per_step / 1e3) / 1e9,
+            "accept_rate": accept_rate, "mean_accept_len": float(g_len.mean()),
+            "timing": {"region_ms": region_ms, "sum_step_ms": sum(step_ms),
+                       "step_ms_median": float(np.median(step_ms)), "k1_ms_median": float(np.median(k1_ms))},
+        }
+        print(json.dumps(line), flush=True)
+    if n > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,195 @@
+/*
+ * spec_verify.h -- C ABI of the B200 (sm_100a) speculative-sampling
+ * verification library (libspecverify.so).
+ *
+ * What it computes.  For each request b of a batch, a drafter proposed
+ * L_b <= k_max tokens x_0 .. x_{L_b-1}.  The target model's logits for the
+ * L_b + 1 positions (and, for a model drafter, the draft model's logits for
+ * the L_b drafted positions) are given.  The library runs the lossless
+ * verification rule described on the pages:
+ *
+ *   - temperature softmax of every used row: p_i = softmax(Z_i / T),
+ *     q_i = softmax(Y_i / T) (or q_i = one-hot at x_i when there are no draft
+ *     logits -- n-gram / suffix-tree drafters supply ids only);
+ *   - draft i is accepted with probability min(1, p_i(x_i) / q_i(x_i)), in
+ *     order, stopping at the first rejection ("AI 开始抄自己的作业——而且抄得理直气壮",
+ *     zhichai.net, section "⚡ 投机解码：让草稿先跑，考官殿后"; and
+ *     "今热点：让AI草稿模型学会"照镜子"" (001ce.com), section
+ *     "先搞懂投机解码在干什么");
+ *   - on a rejection at position j the token is redrawn from the residual
+ *     distribution normalise(max(0, p_j - q_j)) (same NgramRL section);
+ *   - when every draft is accepted, a bonus token is drawn from p at row
+ *     L_b (same page, section "🚰 真正的瓶颈不在算法，在流水线": the step's
+ *     outcome is the pair (j, b));
+ *   - greedy mode replaces sampling by prefix matching against the target's
+ *     argmax ("NgramRL：用Rollout历史加速RL后训练的推测解码新方案",
+ *     kongchang.com, section "一个被忽视的草稿源", glossary entry), ties going
+ *     to the lowest index.
+ *
+ * Readings where the pages are silent: uniforms[b][i] (i < L_b) is the
+ * acceptance draw of draft i and accept iff u < a; uniforms[b][k_max] drives
+ * the final draw; the draw picks the smallest token t whose running weight
+ * sum exceeds u * W (W = total weight); a zero residual mass (only possible
+ * when p == q) falls back to drawing from p_j.
+ *
+ * Layouts (all row-major, "elements" are of the logit dtype):
+ *   target_logits  [B][k_max+1][row_stride]   rows 0..L_b are read
+ *   draft_logits   [B][k_max][row_stride]     rows 0..L_b-1 are read; NULL = one-hot q
+ *   draft_tokens   [B][k_max] int32           entries 0..L_b-1 are read
+ *   draft_lens     [B] int32 in [0, k_max]    NULL = every request uses k_max
+ *   uniforms       [B][k_max+1] float32 in [0, 1)
+ *   out_accept_len [B] int32                  j, the number of accepted drafts
+ *   out_tokens     [B][k_max+1] int32         x_0..x_{j-1}, then the drawn token at
+ *                                             index j, then -1 up to index k_max
+ * Padded rows (beyond L_b) and columns V..row_stride-1 are never read, so
+ * they may hold anything (NaN included).
+ *
+ * Ownership and execution.  Every pointer argument of spec_verify,
+ * spec_verify_ex and spec_verify_stats is DEVICE memory owned by the caller
+ * (spec_verify_host takes host buffers, see there).  The library allocates
+ * nothing.  Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL
+ * = legacy default stream); results are valid once the stream has reached
+ * the call's end.  The workspace needs no initialisation and holds nothing
+ * between calls; two calls that run concurrently need separate workspaces.
+ * The host keeps one small per-device cache of SM count and kernel
+ * attributes.
+ *
+ * Errors.  Argument errors are found on the host before anything is
+ * enqueued and return SV_EINVAL (NULL required pointer, B < 0, k_max < 0,
+ * V < 1, row_stride < V, greedy off with temperature <= 0 or non-finite,
+ * uniforms NULL with greedy off, workspace too small) or SV_EUNSUPPORTED
+ * (k_max > SV_MAX_K, V > SV_MAX_V, unknown dtype).  A failed launch returns
+ * SV_ECUDA.  Values that can only be checked on the device never cause an
+ * out-of-bounds access: a request whose draft_lens entry is outside
+ * [0, k_max] or whose first L_b drafted ids are outside [0, V) gets
+ * out_accept_len = -1 and out_tokens all -1; a request whose statistics were
+ * lost to a device-side wait timeout gets out_accept_len = -2.  NaN or +inf
+ * logits in rows that are read give unspecified (but in-bounds) results.
+ */
+#ifndef SPEC_VERIFY_H
+#define SPEC_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SV_API __attribute__((visibility("default")))
+#else
+#define SV_API
+#endif
+
+#define SV_ABI_VERSION 1
+#define SV_MAX_K 1024      /* largest supported k_max */
+#define SV_MAX_V 393216    /* largest supported vocabulary (8 chunks of 48 Ki) */
+
+typedef enum { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
+
+typedef enum {
+    SV_OK = 0,
+    SV_EINVAL = 1,
+    SV_ECUDA = 2,
+    SV_EUNSUPPORTED = 3
+} sv_status;
+
+/* Problem shape.  row_stride is in elements between consecutive rows
+ * (>= V); 0 means V. */
+typedef struct {
+    int32_t B;
+    int32_t k_max;
+    int32_t V;
+    int32_t dtype; /* sv_dtype of both logit tensors */
+    int64_t row_stride;
+} sv_shape;
+
+/* Which row-statistics kernel to run (spec_verify_ex).  AUTO picks the TMA
+ * bulk-copy pipeline when every row start is 16-byte aligned, else scalar
+ * loads. */
+typedef enum {
+    SV_STATS_AUTO = 0,
+    SV_STATS_TMA = 1,    /* cp.async.bulk + mbarrier ring; needs 16-byte aligned rows */
+    SV_STATS_VEC16 = 2,  /* 16-byte vector loads; needs 16-byte aligned rows */
+    SV_STATS_SCALAR = 3  /* element loads; any alignment */
+} sv_stats_kernel;
+
+typedef struct {
+    int32_t stats_kernel;      /* sv_stats_kernel */
+    int32_t wait_timeout_us;   /* bound on each device-side barrier wait; 0 = 2 s */
+    void *event_stats_begin;   /* cudaEvent_t recorded just before the row-statistics kernel, or NULL */
+    void *event_stats_end;     /* cudaEvent_t recorded just after it, or NULL */
+    int32_t reserved[8];       /* must be zero */
+} sv_options;
+
+/* Bytes of device workspace spec_verify / spec_verify_stats need for this
+ * shape (0 on an invalid shape). */
+SV_API size_t spec_verify_workspace_bytes(const sv_shape *shape);
+
+/* One verification step for the whole batch (see the top of this file).
+ * greedy != 0 selects prefix matching against the target argmax; then
+ * draft_logits, uniforms and temperature are ignored and may be NULL / 0. */
+SV_API sv_status spec_verify(const sv_shape *shape, const void *target_logits,
+                      const void *draft_logits, const int32_t *draft_tokens,
+                      const int32_t *draft_lens, const float *uniforms,
+                      float temperature, int32_t greedy,
+                      int32_t *out_accept_len, int32_t *out_tokens,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* spec_verify with launch options (kernel choice, timing events, wait
+ * bound); opts == NULL is spec_verify. */
+SV_API sv_status spec_verify_ex(const sv_shape *shape, const void *target_logits,
+                         const void *draft_logits, const int32_t *draft_tokens,
+                         const int32_t *draft_lens, const float *uniforms,
+                         float temperature, int32_t greedy,
+                         int32_t *out_accept_len, int32_t *out_tokens,
+                         void *workspace, size_t workspace_bytes, void *stream,
+                         const sv_options *opts);
+
+/* Diagnostic / test hook running the same row-statistics kernel: per used
+ * row the natural-log log-sum-exp of Z/T (out_lse_target [B][k_max+1]) and
+ * Y/T (out_lse_draft [B][k_max], may be NULL), and p_i(x_i), q_i(x_i)
+ * (out_p, out_q [B][k_max]; q = 1 without draft logits).  Entries of rows a
+ * request does not use are NaN; invalid requests get NaN everywhere. */
+SV_API sv_status spec_verify_stats(const sv_shape *shape, const void *target_logits,
+                            const void *draft_logits,
+                            const int32_t *draft_tokens,
+                            const int32_t *draft_lens, float temperature,
+                            float *out_lse_target, float *out_lse_draft,
+                            float *out_p, float *out_q, void *workspace,
+                            size_t workspace_bytes, void *stream,
+                            const sv_options *opts);
+
+/* Bytes of caller-provided device staging memory spec_verify_host needs. */
+SV_API size_t spec_verify_host_staging_bytes(const sv_shape *shape, int32_t has_draft,
+                                      int32_t has_lens);
+
+/* End-to-end form taking HOST buffers (same layouts as spec_verify): copies
+ * the inputs into `device_staging` (cudaMemcpyAsync on `stream`), verifies,
+ * and copies out_accept_len / out_tokens back to the host buffers.  The
+ * copies are asynchronous only when the host buffers are page-locked;
+ * results are valid after the stream is synchronised.  `device_staging`
+ * (spec_verify_host_staging_bytes) and `workspace` are caller-owned device
+ * memory; the library allocates nothing. */
+SV_API sv_status spec_verify_host(const sv_shape *shape, const void *h_target_logits,
+                           const void *h_draft_logits,
+                           const int32_t *h_draft_tokens,
+                           const int32_t *h_draft_lens, const float *h_uniforms,
+                           float temperature, int32_t greedy,
+                           int32_t *h_out_accept_len, int32_t *h_out_tokens,
+                           void *device_staging, size_t staging_bytes,
+                           void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Static description of a status code. */
+SV_API const char *spec_verify_status_string(sv_status status);
+
+/* SV_ABI_VERSION of the built library. */
+SV_API int32_t spec_verify_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEC_VERIFY_H */

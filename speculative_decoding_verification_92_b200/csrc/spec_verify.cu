@@ -1,0 +1,415 @@
+// spec_verify.cu -- host side of libspecverify.so: argument checks, the
+// chunk plan, launches of K1 (row statistics) and K2 (scan + draw), and the
+// extern "C" entry points declared in include/spec_verify.h.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "spec_verify.h"
+#include "sv_common.cuh"
+#include "sv_row_stats.cuh"
+#include "sv_verify_draw.cuh"
+
+namespace sv {
+namespace {
+
+constexpr int kTmaConsumerWarps = SV_TMA_CONSUMER_WARPS;
+constexpr int kTmaStages = SV_TMA_STAGES;
+constexpr int kTmaCtasPerSm = SV_TMA_CTAS_PER_SM;
+constexpr int kLdgThreads = 256;
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int max_smem_optin = 0;
+    bool ready = false;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+cudaError_t device_info(DeviceInfo** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        d.ready = true;
+    }
+    *out = &d;
+    return cudaSuccess;
+}
+
+// Opt a kernel into `bytes` of dynamic shared memory (idempotent per device).
+template <typename Kernel>
+cudaError_t allow_smem(Kernel k, size_t bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+struct Plan {
+    int C = 1;       // chunks per row
+    int CE = 8;      // elements per chunk (multiple of 8)
+    int es = 4;      // element size
+    int64_t stride = 0;
+};
+
+// Rows are cut into at most kMaxChunks chunks of about 32 KiB; a chunk starts
+// on a 16-byte boundary of an aligned row.
+Plan make_plan(const sv_shape& s) {
+    Plan p;
+    p.es = s.dtype == SV_BF16 ? 2 : 4;
+    p.stride = s.row_stride ? s.row_stride : s.V;
+    const int64_t row_bytes = int64_t(s.V) * p.es;
+    int c = static_cast<int>((row_bytes + 32767) / 32768);
+    c = c < 1 ? 1 : (c > kMaxChunks ? kMaxChunks : c);
+    int ce = (s.V + c - 1) / c;
+    ce = (ce + 7) & ~7;
+    p.CE = ce;
+    p.C = (s.V + ce - 1) / ce;
+    return p;
+}
+
+bool shape_ok(const sv_shape* s, sv_status* why) {
+    if (!s) { *why = SV_EINVAL; return false; }
+    if (s->B < 0 || s->k_max < 0 || s->V < 1) { *why = SV_EINVAL; return false; }
+    if (s->dtype != SV_F32 && s->dtype != SV_BF16) { *why = SV_EUNSUPPORTED; return false; }
+    if (s->k_max > SV_MAX_K || s->V > SV_MAX_V) { *why = SV_EUNSUPPORTED; return false; }
+    const int64_t stride = s->row_stride ? s->row_stride : s->V;
+    if (stride < s->V) { *why = SV_EINVAL; return false; }
+    return true;
+}
+
+size_t workspace_bytes_for(const sv_shape& s, const Plan& p) {
+    const size_t n = size_t(s.B) * size_t(2 * s.k_max + 1) * size_t(p.C) * sizeof(float2);
+    return (n + 255) & ~size_t(255);
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+template <typename T, bool kGreedy>
+cudaError_t launch_stats(const StatsParams& base, int B, int variant, const DeviceInfo& dev, cudaStream_t st) {
+    for (int b0 = 0; b0 < B; b0 += kMaxRequestsPerLaunch) {
+        StatsParams prm = base;
+        prm.b0 = b0;
+        prm.nB = B - b0 < kMaxRequestsPerLaunch ? B - b0 : kMaxRequestsPerLaunch;
+        const int rows_max = prm.use_draft ? 2 * prm.k_max + 1 : prm.k_max + 1;
+        const int64_t items_upper = int64_t(prm.nB) * rows_max * prm.C;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 0;
+        cudaError_t e;
+        if (variant == SV_STATS_TMA) {
+            auto k = row_stats_tma_kernel<T, kGreedy, kTmaConsumerWarps, kTmaStages>;
+            const size_t smem = TmaSmem<kTmaConsumerWarps, kTmaStages>::bytes(prm.nB);
+            if ((e = allow_smem(k, smem)) != cudaSuccess) return e;
+            const int64_t cap = int64_t(dev.sm_count) * kTmaCtasPerSm;
+            const int64_t grid = items_upper < cap ? items_upper : cap;
+            cfg.gridDim = dim3(static_cast<unsigned>(grid));
+            cfg.blockDim = dim3((kTmaConsumerWarps + 1) * 32);
+            cfg.dynamicSmemBytes = smem;
+            e = cudaLaunchKernelEx(&cfg, k, prm);
+        } else {
+            auto k = variant == SV_STATS_VEC16 ? row_stats_ldg_kernel<T, kGreedy, true, kLdgThreads>
+                                               : row_stats_ldg_kernel<T, kGreedy, false, kLdgThreads>;
+            const size_t smem = 4 * size_t(prm.nB + 1);
+            if ((e = allow_smem(k, smem)) != cudaSuccess) return e;
+            int per_sm = 0;
+            if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kLdgThreads, smem)) != cudaSuccess)
+                return e;
+            if (per_sm < 1) per_sm = 1;
+            const int64_t cap = int64_t(dev.sm_count) * per_sm;
+            const int64_t grid = items_upper < cap ? items_upper : cap;
+            cfg.gridDim = dim3(static_cast<unsigned>(grid));
+            cfg.blockDim = dim3(kLdgThreads);
+            cfg.dynamicSmemBytes = smem;
+            e = cudaLaunchKernelEx(&cfg, k, prm);
+        }
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t launch_draw(const DrawParams& base, int B, cudaStream_t st) {
+    auto k = verify_draw_kernel<T>;
+    const size_t smem = draw_smem_bytes(base.CE, base.k_max);
+    cudaError_t e = allow_smem(k, smem);
+    if (e != cudaSuccess) return e;
+    for (int b0 = 0; b0 < B; b0 += 65535) {
+        DrawParams prm = base;
+        prm.b0 = b0;
+        const int nB = B - b0 < 65535 ? B - b0 : 65535;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(prm.C);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(static_cast<unsigned>(prm.C), static_cast<unsigned>(nB));
+        cfg.blockDim = dim3(kDrawThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&cfg, k, prm)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+struct Call {
+    const sv_shape* shape;
+    const void* target;
+    const void* draft;
+    const int32_t* tokens;
+    const int32_t* lens;
+    const float* uniforms;
+    float temperature;
+    int greedy;
+    int32_t* out_len;
+    int32_t* out_tokens;
+    float* out_lse_t;
+    float* out_lse_d;
+    float* out_p;
+    float* out_q;
+    void* workspace;
+    size_t workspace_bytes;
+    cudaStream_t stream;
+    const sv_options* opts;
+    bool stats_only;
+};
+
+template <typename T>
+sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int variant, bool rows_aligned) {
+    const sv_shape& s = *a.shape;
+    const bool greedy = a.greedy && !a.stats_only;
+    StatsParams sp{};
+    sp.target = static_cast<const unsigned char*>(a.target);
+    sp.draft = static_cast<const unsigned char*>(a.draft);
+    sp.lens = a.lens;
+    sp.partials = static_cast<float2*>(a.workspace);
+    sp.k_max = s.k_max;
+    sp.V = s.V;
+    sp.row_stride = plan.stride;
+    sp.C = plan.C;
+    sp.CE = plan.CE;
+    sp.scale = greedy ? 1.f : static_cast<float>(kLog2e / static_cast<double>(a.temperature));
+    sp.use_draft = (a.draft != nullptr && !greedy) ? 1 : 0;
+    const int tmo = a.opts ? a.opts->wait_timeout_us : 0;
+    sp.timeout_ns = tmo > 0 ? uint64_t(tmo) * 1000ull : kDefaultTimeoutNs;
+
+    cudaError_t e = cudaSuccess;
+    if (a.opts && a.opts->event_stats_begin)
+        if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_begin), a.stream)) != cudaSuccess)
+            return SV_ECUDA;
+    e = greedy ? launch_stats<T, true>(sp, s.B, variant, dev, a.stream)
+               : launch_stats<T, false>(sp, s.B, variant, dev, a.stream);
+    if (e != cudaSuccess) return SV_ECUDA;
+    if (a.opts && a.opts->event_stats_end)
+        if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_end), a.stream)) != cudaSuccess)
+            return SV_ECUDA;
+
+    DrawParams dp{};
+    dp.target = sp.target;
+    dp.draft = greedy ? nullptr : sp.draft;
+    dp.tokens = a.tokens;
+    dp.lens = a.lens;
+    dp.uniforms = a.uniforms;
+    dp.partials = sp.partials;
+    dp.out_len = a.out_len;
+    dp.out_tokens = a.out_tokens;
+    dp.out_lse_t = a.out_lse_t;
+    dp.out_lse_d = a.out_lse_d;
+    dp.out_p = a.out_p;
+    dp.out_q = a.out_q;
+    dp.k_max = s.k_max;
+    dp.V = s.V;
+    dp.row_stride = plan.stride;
+    dp.C = plan.C;
+    dp.CE = plan.CE;
+    dp.scale = sp.scale;
+    dp.greedy = greedy ? 1 : 0;
+    dp.stats_only = a.stats_only ? 1 : 0;
+    dp.rows_aligned = rows_aligned ? 1 : 0;
+    e = launch_draw<T>(dp, s.B, a.stream);
+    return e == cudaSuccess ? SV_OK : SV_ECUDA;
+}
+
+sv_status run(const Call& a) {
+    sv_status why = SV_OK;
+    if (!shape_ok(a.shape, &why)) return why;
+    const sv_shape& s = *a.shape;
+    if (a.opts) {
+        for (int i = 0; i < 8; ++i)
+            if (a.opts->reserved[i] != 0) return SV_EINVAL;
+        if (a.opts->stats_kernel < SV_STATS_AUTO || a.opts->stats_kernel > SV_STATS_SCALAR) return SV_EINVAL;
+        if (a.opts->wait_timeout_us < 0) return SV_EINVAL;
+    }
+    if (s.B == 0) return SV_OK;
+    const bool greedy = a.greedy && !a.stats_only;
+    if (!a.target) return SV_EINVAL;
+    if (s.k_max > 0 && !a.tokens) return SV_EINVAL;
+    if (a.stats_only) {
+        if (!a.out_lse_t) return SV_EINVAL;
+    } else {
+        if (!a.out_len || !a.out_tokens) return SV_EINVAL;
+    }
+    if (!greedy) {
+        if (!(a.temperature > 0.f) || !std::isfinite(a.temperature)) return SV_EINVAL;
+        if (!a.stats_only && !a.uniforms) return SV_EINVAL;
+    }
+    const Plan plan = make_plan(s);
+    if (!a.workspace || a.workspace_bytes < workspace_bytes_for(s, plan)) return SV_EINVAL;
+    if (!aligned16(a.workspace)) return SV_EINVAL;
+
+    DeviceInfo* dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return SV_ECUDA;
+    if (draw_smem_bytes(plan.CE, s.k_max) + 2048 > size_t(dev->max_smem_optin)) return SV_EUNSUPPORTED;
+
+    // Kernel choice: the bulk-copy and vector paths need every row start on a
+    // 16-byte boundary.
+    const bool rows_aligned = aligned16(a.target) && (a.draft == nullptr || greedy || aligned16(a.draft)) &&
+                              ((plan.stride * plan.es) % 16 == 0);
+    int variant = a.opts ? a.opts->stats_kernel : SV_STATS_AUTO;
+    if (variant == SV_STATS_AUTO) variant = rows_aligned ? SV_STATS_TMA : SV_STATS_SCALAR;
+    if ((variant == SV_STATS_TMA || variant == SV_STATS_VEC16) && !rows_aligned) return SV_EINVAL;
+
+    return s.dtype == SV_BF16 ? run_typed<bf16_bits>(a, plan, *dev, variant, rows_aligned)
+                              : run_typed<float>(a, plan, *dev, variant, rows_aligned);
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+struct HostLayout {
+    size_t target, draft, tokens, lens, uniforms, out_len, out_tokens, total;
+};
+
+HostLayout host_layout(const sv_shape& s, bool has_draft, bool has_lens) {
+    const Plan plan = make_plan(s);
+    HostLayout h{};
+    const size_t B = size_t(s.B), K = size_t(s.k_max), es = size_t(plan.es), st = size_t(plan.stride);
+    size_t off = 0;
+    h.target = off; off += align256(B * (K + 1) * st * es);
+    h.draft = off; off += has_draft ? align256(B * K * st * es) : 0;
+    h.tokens = off; off += align256(B * K * 4);
+    h.lens = off; off += has_lens ? align256(B * 4) : 0;
+    h.uniforms = off; off += align256(B * (K + 1) * 4);
+    h.out_len = off; off += align256(B * 4);
+    h.out_tokens = off; off += align256(B * (K + 1) * 4);
+    h.total = off;
+    return h;
+}
+
+}  // namespace
+}  // namespace sv
+
+extern "C" {
+
+size_t spec_verify_workspace_bytes(const sv_shape* shape) {
+    sv_status why;
+    if (!sv::shape_ok(shape, &why)) return 0;
+    return sv::workspace_bytes_for(*shape, sv::make_plan(*shape));
+}
+
+sv_status spec_verify_ex(const sv_shape* shape, const void* target_logits, const void* draft_logits,
+                         const int32_t* draft_tokens, const int32_t* draft_lens, const float* uniforms,
+                         float temperature, int32_t greedy, int32_t* out_accept_len, int32_t* out_tokens,
+                         void* workspace, size_t workspace_bytes, void* stream, const sv_options* opts) {
+    sv::Call a{shape,      target_logits, draft_logits, draft_tokens,   draft_lens,
+               uniforms,   temperature,   greedy != 0,  out_accept_len, out_tokens,
+               nullptr,    nullptr,       nullptr,      nullptr,        workspace,
+               workspace_bytes, static_cast<cudaStream_t>(stream), opts, false};
+    return sv::run(a);
+}
+
+sv_status spec_verify(const sv_shape* shape, const void* target_logits, const void* draft_logits,
+                      const int32_t* draft_tokens, const int32_t* draft_lens, const float* uniforms,
+                      float temperature, int32_t greedy, int32_t* out_accept_len, int32_t* out_tokens,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    return spec_verify_ex(shape, target_logits, draft_logits, draft_tokens, draft_lens, uniforms, temperature,
+                          greedy, out_accept_len, out_tokens, workspace, workspace_bytes, stream, nullptr);
+}
+
+sv_status spec_verify_stats(const sv_shape* shape, const void* target_logits, const void* draft_logits,
+                            const int32_t* draft_tokens, const int32_t* draft_lens, float temperature,
+                            float* out_lse_target, float* out_lse_draft, float* out_p, float* out_q,
+                            void* workspace, size_t workspace_bytes, void* stream, const sv_options* opts) {
+    sv::Call a{shape,          target_logits, draft_logits, draft_tokens, draft_lens,
+               nullptr,        temperature,   false,        nullptr,      nullptr,
+               out_lse_target, out_lse_draft, out_p,        out_q,        workspace,
+               workspace_bytes, static_cast<cudaStream_t>(stream), opts, true};
+    return sv::run(a);
+}
+
+size_t spec_verify_host_staging_bytes(const sv_shape* shape, int32_t has_draft, int32_t has_lens) {
+    sv_status why;
+    if (!sv::shape_ok(shape, &why)) return 0;
+    return sv::host_layout(*shape, has_draft != 0, has_lens != 0).total;
+}
+
+sv_status spec_verify_host(const sv_shape* shape, const void* h_target_logits, const void* h_draft_logits,
+                           const int32_t* h_draft_tokens, const int32_t* h_draft_lens, const float* h_uniforms,
+                           float temperature, int32_t greedy, int32_t* h_out_accept_len, int32_t* h_out_tokens,
+                           void* device_staging, size_t staging_bytes, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    sv_status why;
+    if (!sv::shape_ok(shape, &why)) return why;
+    const sv_shape& s = *shape;
+    if (s.B == 0) return SV_OK;
+    const bool has_draft = h_draft_logits != nullptr && !greedy;
+    const bool has_lens = h_draft_lens != nullptr;
+    const sv::HostLayout h = sv::host_layout(s, has_draft, has_lens);
+    if (!device_staging || staging_bytes < h.total || !sv::aligned16(device_staging)) return SV_EINVAL;
+    if (!h_target_logits || !h_out_accept_len || !h_out_tokens) return SV_EINVAL;
+    if (s.k_max > 0 && !h_draft_tokens) return SV_EINVAL;
+    if (!greedy && !h_uniforms) return SV_EINVAL;
+    const sv::Plan plan = sv::make_plan(s);
+    const size_t B = size_t(s.B), K = size_t(s.k_max), es = size_t(plan.es), st = size_t(plan.stride);
+    unsigned char* base = static_cast<unsigned char*>(device_staging);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    auto h2d = [&](size_t off, const void* src, size_t n) {
+        return n ? cudaMemcpyAsync(base + off, src, n, cudaMemcpyHostToDevice, cs) : cudaSuccess;
+    };
+    cudaError_t e = h2d(h.target, h_target_logits, B * (K + 1) * st * es);
+    if (e == cudaSuccess && has_draft) e = h2d(h.draft, h_draft_logits, B * K * st * es);
+    if (e == cudaSuccess && K) e = h2d(h.tokens, h_draft_tokens, B * K * 4);
+    if (e == cudaSuccess && has_lens) e = h2d(h.lens, h_draft_lens, B * 4);
+    if (e == cudaSuccess && !greedy) e = h2d(h.uniforms, h_uniforms, B * (K + 1) * 4);
+    if (e != cudaSuccess) return SV_ECUDA;
+    sv_status r = spec_verify(shape, base + h.target, has_draft ? base + h.draft : nullptr,
+                              reinterpret_cast<const int32_t*>(base + h.tokens),
+                              has_lens ? reinterpret_cast<const int32_t*>(base + h.lens) : nullptr,
+                              greedy ? nullptr : reinterpret_cast<const float*>(base + h.uniforms), temperature,
+                              greedy, reinterpret_cast<int32_t*>(base + h.out_len),
+                              reinterpret_cast<int32_t*>(base + h.out_tokens), workspace, workspace_bytes, stream);
+    if (r != SV_OK) return r;
+    e = cudaMemcpyAsync(h_out_accept_len, base + h.out_len, B * 4, cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(h_out_tokens, base + h.out_tokens, B * (K + 1) * 4, cudaMemcpyDeviceToHost, cs);
+    return e == cudaSuccess ? SV_OK : SV_ECUDA;
+}
+
+const char* spec_verify_status_string(sv_status status) {
+    switch (status) {
+        case SV_OK: return "ok";
+        case SV_EINVAL: return "invalid argument";
+        case SV_ECUDA: return "CUDA error";
+        case SV_EUNSUPPORTED: return "unsupported shape or dtype";
+    }
+    return "unknown status";
+}
+
+int32_t spec_verify_abi_version(void) { return SV_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+"""The C-ABI library on a machine without a GPU: it builds, loads, exports
+every symbol include/*.h declares, and rejects bad arguments on the host
+before any CUDA call.  No kernel is launched here."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import speculative_decoding_verification_92_b200 as sv
+from speculative_decoding_verification_92_b200 import _Options, _Shape, Status
+
+ROOT = Path(__file__).resolve().parents[1]
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails before touching it
+
+
+def declared_symbols():
+    names = []
+    for h in sorted((ROOT / "include").glob("*.h")):
+        text = h.read_text()
+        names += re.findall(r"SV_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = sv.library()
+    names = declared_symbols()
+    assert len(names) >= 8, names
+    for name in names:
+        assert hasattr(lib, name), f"{name} is declared in include/ but not exported"
+    assert sv.abi_version() == 1
+
+
+def test_status_strings():
+    lib = sv.library()
+    for code in Status:
+        s = lib.spec_verify_status_string(int(code))
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.spec_verify_status_string(99) == b"unknown status"
+
+
+def plan_chunks(V, es):
+    c = max(1, min(8, -(-V * es // 32768)))
+    ce = -(-V // c)
+    ce = (ce + 7) & ~7
+    return -(-V // ce), ce
+
+
+@pytest.mark.parametrize("B,k,V,dt", [(64, 8, 151936, sv.BF16), (256, 12, 128256, sv.F32),
+                                      (4, 4, 1000, sv.F32), (3, 0, 5, sv.BF16), (0, 3, 100, sv.F32)])
+def test_workspace_bytes(B, k, V, dt):
+    C, _ = plan_chunks(V, 2 if dt == sv.BF16 else 4)
+    want = B * (2 * k + 1) * C * 8
+    want = (want + 255) // 256 * 256
+    assert sv.workspace_bytes(B, k, V, dt) == want
+
+
+def test_workspace_bytes_invalid_shape():
+    lib = sv.library()
+    assert lib.spec_verify_workspace_bytes(None) == 0
+    assert sv.workspace_bytes(4, 4, 0, sv.F32) == 0
+    assert sv.workspace_bytes(4, -1, 10, sv.F32) == 0
+    assert sv.workspace_bytes(4, 4, 10, 9) == 0
+    assert sv.workspace_bytes(4, 4, 10, sv.F32, row_stride=5) == 0
+
+
+def call(shape=None, target=FAKE, draft=None, tokens=FAKE, lens=None, uniforms=FAKE, T=1.0, greedy=0,
+         out_len=FAKE, out_tok=FAKE, ws=FAKE, ws_bytes=1 << 30, opts=None):
+    lib = sv.library()
+    if shape is None:
+        shape = _Shape(4, 4, 1000, sv.F32, 0)
+    return lib.spec_verify_ex(ctypes.byref(shape) if shape is not False else None, target, draft, tokens, lens,
+                              uniforms, T, greedy, out_len, out_tok, ws, ws_bytes, None,
+                              ctypes.byref(opts) if opts is not None else None)
+
+
+@pytest.mark.parametrize("kwargs,want", [
+    (dict(shape=False), Status.EINVAL),
+    (dict(shape=_Shape(4, 4, 0, sv.F32, 0)), Status.EINVAL),
+    (dict(shape=_Shape(-1, 4, 10, sv.F32, 0)), Status.EINVAL),
+    (dict(shape=_Shape(4, -2, 10, sv.F32, 0)), Status.EINVAL),
+    (dict(shape=_Shape(4, 4, 10, sv.F32, 9)), Status.EINVAL),
+    (dict(shape=_Shape(4, 4, 10, 5, 0)), Status.EUNSUPPORTED),
+    (dict(shape=_Shape(4, 1025, 10, sv.F32, 0)), Status.EUNSUPPORTED),
+    (dict(shape=_Shape(4, 4, 393217, sv.F32, 0)), Status.EUNSUPPORTED),
+    (dict(target=None), Status.EINVAL),
+    (dict(tokens=None), Status.EINVAL),
+    (dict(out_len=None), Status.EINVAL),
+    (dict(out_tok=None), Status.EINVAL),
+    (dict(uniforms=None), Status.EINVAL),
+    (dict(T=0.0), Status.EINVAL),
+    (dict(T=-1.0), Status.EINVAL),
+    (dict(T=float("nan")), Status.EINVAL),
+    (dict(T=float("inf")), Status.EINVAL),
+    (dict(ws=None), Status.EINVAL),
+    (dict(ws_bytes=8), Status.EINVAL),
+    (dict(ws=FAKE + 4), Status.EINVAL),
+])
+def test_argument_errors_before_any_launch(kwargs, want):
+    assert call(**kwargs) == want
+
+
+def test_bad_options():
+    o = _Options()
+    o.reserved[3] = 1
+    assert call(opts=o) == Status.EINVAL
+    o = _Options()
+    o.stats_kernel = 7
+    assert call(opts=o) == Status.EINVAL
+    o = _Options()
+    o.wait_timeout_us = -5
+    assert call(opts=o) == Status.EINVAL
+
+
+def test_greedy_needs_no_uniforms_or_temperature_and_empty_batch_is_ok():
+    # greedy: uniforms NULL and T = 0 pass validation; with B = 0 nothing is launched
+    assert call(shape=_Shape(0, 4, 1000, sv.F32, 0), uniforms=None, T=0.0, greedy=1) == Status.OK
+    assert call(shape=_Shape(0, 4, 1000, sv.F32, 0)) == Status.OK
+
+
+def test_valid_call_without_gpu_reports_cuda_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert call() == Status.ECUDA
+
+
+def test_stats_and_host_entry_points_validate():
+    lib = sv.library()
+    shape = _Shape(4, 4, 1000, sv.F32, 0)
+    # stats: missing lse output
+    assert lib.spec_verify_stats(ctypes.byref(shape), FAKE, None, FAKE, None, 1.0, None, None, None, None,
+                                 FAKE, 1 << 20, None, None) == Status.EINVAL
+    # host form: staging too small
+    n = lib.spec_verify_host_staging_bytes(ctypes.byref(shape), 1, 0)
+    assert n >= 4 * 5 * 1000 * 4 + 4 * 4 * 1000 * 4
+    assert lib.spec_verify_host(ctypes.byref(shape), FAKE, FAKE, FAKE, None, FAKE, 1.0, 0, FAKE, FAKE,
+                                FAKE, n - 1, FAKE, 1 << 20, None) == Status.EINVAL
+
+
+def test_python_binding_rejects_host_tensors():
+    import torch
+    t = torch.zeros(2, 3, 10)
+    with pytest.raises(ValueError):
+        sv.spec_verify(t, None, torch.zeros(2, 2, dtype=torch.int32), None, torch.zeros(2, 3))
