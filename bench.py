@@ -74,6 +74,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--greedy", action="store_true", help="time the greedy (prefix-match) form instead")
+    ap.add_argument("--event-every", type=int, default=16,
+                    help="bracket the row-statistics kernel with events on every N-th timed step")
     return ap.parse_args()
 
 
@@ -349,8 +351,12 @@ def run_ours_impl(args):
     for _ in range(W):
         step()
     torch.cuda.synchronize()
-    step_ev = [(new_event(), new_event()) for _ in range(K)]
-    k1_ev = [(new_event(), new_event()) for _ in range(K)]
+    # Events cost a few microseconds each on the stream, so only every
+    # EVENT_EVERY-th step brackets the row-statistics kernel; steps are timed
+    # individually only when the L2 is flushed between them.
+    every = max(1, args.event_every)
+    k1_ev = {i: (new_event(), new_event()) for i in range(0, K, every)}
+    step_ev = [(new_event(), new_event()) for _ in range(K)] if flush_buf is not None else None
     g0, g1 = new_event(), new_event()
     torch.cuda.synchronize()
 
@@ -361,16 +367,17 @@ def run_ours_impl(args):
         for i in range(K):
             if flush_buf is not None:
                 flush_buf.fill_(i)
-            step_ev[i][0].record(stream)
-            step(events=k1_ev[i])
-            step_ev[i][1].record(stream)
+                step_ev[i][0].record(stream)
+            step(events=k1_ev.get(i))
+            if flush_buf is not None:
+                step_ev[i][1].record(stream)
         g1.record(stream)
         torch.cuda.synchronize()
     barrier()
 
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    k1_ms = [a.elapsed_time(b) for a, b in k1_ev]
+    k1_ms = [a.elapsed_time(b) for a, b in k1_ev.values()]
     region_ms = g0.elapsed_time(g1)
+    step_ms = [a.elapsed_time(b) for a, b in step_ev] if step_ev is not None else [region_ms / K]
     t_rank = sum(step_ms) if flush_buf is not None else region_ms
     t_max = t_rank
     if n > 1:
@@ -464,8 +471,8 @@ def run_ours_impl(args):
             "cpu_baseline": cpu, "clocks": clocks.summary(),
             "hbm_gbs": alg / (ms_per_step / 1e3) / 1e9,
             "accept_rate": accept_rate, "mean_accept_len": float(g_len.mean()),
-            "timing": {"region_ms": region_ms, "sum_step_ms": sum(step_ms),
-                       "step_ms_median": float(np.median(step_ms)), "k1_ms_median": float(np.median(k1_ms))},
+            "timing": {"region_ms": region_ms, "k1_event_samples": len(k1_ms), "k1_event_every": every,
+                       "k1_ms_median": float(np.median(k1_ms))},
         }
         print(json.dumps(line), flush=True)
     if n > 1:

@@ -20,6 +20,10 @@ constexpr int kTmaConsumerWarps = SV_TMA_CONSUMER_WARPS;
 constexpr int kTmaStages = SV_TMA_STAGES;
 constexpr int kTmaCtasPerSm = SV_TMA_CTAS_PER_SM;
 constexpr int kLdgThreads = 256;
+// Draw-kernel grid: about SV_DRAW_WAVES waves of 2 CTAs per SM.
+#ifndef SV_DRAW_WAVES
+#define SV_DRAW_WAVES 1
+#endif
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 
@@ -143,26 +147,32 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
 
 template <typename T>
 cudaError_t launch_draw(const DrawParams& base, int B, cudaStream_t st) {
+    // A request's cluster has C2 = ceil(C / R) CTAs; R is chosen so that the
+    // whole batch is about SV_DRAW_WAVES waves of CTAs (2 per SM).
     auto k = verify_draw_kernel<T>;
-    const size_t smem = draw_smem_bytes(base.CE, base.k_max);
+    const size_t smem = draw_smem_bytes(base.C, base.k_max);
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return e;
     for (int b0 = 0; b0 < B; b0 += 65535) {
         DrawParams prm = base;
         prm.b0 = b0;
         const int nB = B - b0 < 65535 ? B - b0 : 65535;
+        const int C2 = (prm.C + prm.R - 1) / prm.R;
         cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(prm.C);
+        attr[0].val.clusterDim.x = static_cast<unsigned>(C2);
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3(static_cast<unsigned>(prm.C), static_cast<unsigned>(nB));
+        // programmatic dependent of the row-statistics kernel launched just before
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.gridDim = dim3(static_cast<unsigned>(C2), static_cast<unsigned>(nB));
         cfg.blockDim = dim3(kDrawThreads);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         if ((e = cudaLaunchKernelEx(&cfg, k, prm)) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -242,6 +252,11 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     dp.greedy = greedy ? 1 : 0;
     dp.stats_only = a.stats_only ? 1 : 0;
     dp.rows_aligned = rows_aligned ? 1 : 0;
+    {
+        const int64_t target_ctas = int64_t(dev.sm_count) * 2 * SV_DRAW_WAVES;
+        int64_t r = (int64_t(plan.C) * s.B + target_ctas - 1) / target_ctas;
+        dp.R = static_cast<int>(r < 1 ? 1 : (r > plan.C ? plan.C : r));
+    }
     e = launch_draw<T>(dp, s.B, a.stream);
     return e == cudaSuccess ? SV_OK : SV_ECUDA;
 }
@@ -275,7 +290,7 @@ sv_status run(const Call& a) {
 
     DeviceInfo* dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return SV_ECUDA;
-    if (draw_smem_bytes(plan.CE, s.k_max) + 2048 > size_t(dev->max_smem_optin)) return SV_EUNSUPPORTED;
+    if (draw_smem_bytes(plan.C, s.k_max) + 4096 > size_t(dev->max_smem_optin)) return SV_EUNSUPPORTED;
 
     // Kernel choice: the bulk-copy and vector paths need every row start on a
     // 16-byte boundary.

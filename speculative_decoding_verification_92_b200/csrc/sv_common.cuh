@@ -57,25 +57,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// Packed pairs (Blackwell f32x2 arithmetic and bf16x2 max).
-__device__ __forceinline__ uint64_t pack2(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void unpack2(uint64_t v, float& a, float& b) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
+// Packed bf16x2 maximum of two words (two elements per instruction).
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -175,6 +157,19 @@ __device__ __forceinline__ MS ms_merge(MS a, MS b) {
     const float m = fmaxf(a.m, b.m);
     if (m == -INFINITY) return MS{-INFINITY, 0.f};
     return MS{m, a.s * ex2_approx(a.m - m) + b.s * ex2_approx(b.m - m)};
+}
+
+// Warp reduction of (m, s) pairs with one ex2 per lane: the warp maximum
+// first, then every lane rescales its own sum to it and the sums are added.
+__device__ __forceinline__ MS warp_merge_ms_maxfirst(MS v) {
+    float m = v.m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (m == -INFINITY) return MS{-INFINITY, 0.f};
+    float s = v.s * ex2_approx(v.m - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return MS{m, s};
 }
 
 __device__ __forceinline__ MS warp_merge_ms(MS v) {

@@ -24,6 +24,24 @@
 
 #include "sv_common.cuh"
 
+// Ring geometry of the bulk-copy variant (compile-time; defaults tuned on B200).
+#ifndef SV_STAGE_BYTES
+#define SV_STAGE_BYTES 16384
+#endif
+#ifndef SV_TMA_CONSUMER_WARPS
+#define SV_TMA_CONSUMER_WARPS 4
+#endif
+#ifndef SV_TMA_STAGES
+#define SV_TMA_STAGES 3
+#endif
+#ifndef SV_TMA_CTAS_PER_SM
+#define SV_TMA_CTAS_PER_SM 4
+#endif
+// 16-byte vectors per thread in flight in the vector-load variant.
+#ifndef SV_LDG_UNROLL
+#define SV_LDG_UNROLL 4
+#endif
+
 namespace sv {
 
 struct StatsParams {
@@ -181,16 +199,17 @@ template <> struct Acc<true> {
     }
 };
 
-// Fold K 16-byte vectors of raw logits into a sampling accumulator with the
-// packed Blackwell forms: for bf16 the row max comes from max.bf16x2 on the
-// stored words (no unpacking), the exponent arguments fma(z, scale, -M) and
-// the sums run as f32x2 pairs, one ex2 per element.  Absent vectors must be
-// passed as -inf (bf16 words 0xff80ff80, fp32 0xff800000).
+// Fold K 16-byte vectors of raw logits into a sampling accumulator.  The
+// row maximum of bf16 data comes from max.bf16x2 on the stored words (half an
+// instruction per element, no unpacking); then each element costs one
+// integer unpack (bf16), one FFMA for z * scale - M, one ex2 and one FADD into
+// one of four independent partial sums.  Absent vectors must be passed as
+// -inf (bf16 words 0xff80ff80, fp32 0xff800000).
 constexpr uint32_t kBf16NegInfPair = 0xff80ff80u;
 constexpr uint32_t kF32NegInfBits = 0xff800000u;
 
 template <typename T, int K>
-__device__ __forceinline__ void fold_vectors(Acc<false>& acc, const uint4 (&v)[K], float scale, uint64_t scale2) {
+__device__ __forceinline__ void fold_vectors(Acc<false>& acc, const uint4 (&v)[K], float scale) {
     constexpr int NW = 4 * K;
     uint32_t w[NW];
 #pragma unroll
@@ -219,24 +238,46 @@ __device__ __forceinline__ void fold_vectors(Acc<false>& acc, const uint4 (&v)[K
     }
     const float M = fmaxf(acc.ms.m, zmax * scale);
     if (M == -INFINITY) return;
-    const uint64_t negM2 = pack2(-M, -M);
-    constexpr int NP = Logit<T>::kSize == 2 ? NW : NW / 2;  // element pairs
-    uint64_t e2[NP];
+    const float negM = -M;
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < NP; ++i) {
-        const uint64_t t = Logit<T>::kSize == 2 ? pack2(bf16_lo(w[i]), bf16_hi(w[i]))
-                                                 : pack2(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
-        float a, b;
-        unpack2(fma2(t, scale2, negM2), a, b);
-        e2[i] = pack2(ex2_approx(a), ex2_approx(b));
+    for (int i = 0; i < NW; ++i) {
+        if constexpr (Logit<T>::kSize == 2) {
+            s[(2 * i) & 3] += ex2_approx(fmaf(bf16_lo(w[i]), scale, negM));
+            s[(2 * i + 1) & 3] += ex2_approx(fmaf(bf16_hi(w[i]), scale, negM));
+        } else {
+            s[i & 3] += ex2_approx(fmaf(__uint_as_float(w[i]), scale, negM));
+        }
     }
+    acc.ms = MS{M, fmaf(acc.ms.s, ex2_approx(acc.ms.m - M), (s[0] + s[1]) + (s[2] + s[3]))};
+}
+
+// Fold only the first `nv` (0 <= nv <= K) of K vectors: one fold with a
+// compile-time count per possible nv, so no ex2 is spent on absent elements
+// (the partial stage or batch at the end of each item).
+template <typename T, int K, int N>
+__device__ __forceinline__ void fold_prefix(Acc<false>& acc, const uint4 (&v)[K], float scale) {
+    uint4 part[N];
 #pragma unroll
-    for (int d = 1; d < NP; d <<= 1)
-#pragma unroll
-        for (int i = 0; i + d < NP; i += 2 * d) e2[i] = add2(e2[i], e2[i + d]);
-    float a, b;
-    unpack2(e2[0], a, b);
-    acc.ms = MS{M, fmaf(acc.ms.s, ex2_approx(acc.ms.m - M), a + b)};
+    for (int k = 0; k < N; ++k) part[k] = v[k];
+    fold_vectors<T, N>(acc, part, scale);
+}
+
+template <typename T, int K, int N>
+__device__ __forceinline__ void fold_prefix_select(Acc<false>& acc, const uint4 (&v)[K], int nv, float scale) {
+    if constexpr (N >= 1) {
+        if (nv == N) {
+            fold_prefix<T, K, N>(acc, v, scale);
+            return;
+        }
+        fold_prefix_select<T, K, N - 1>(acc, v, nv, scale);
+    }
+}
+
+template <typename T, int K>
+__device__ __forceinline__ void fold_vectors_count(Acc<false>& acc, const uint4 (&v)[K], int nv, float scale) {
+    if (nv >= K) fold_vectors<T, K>(acc, v, scale);
+    else fold_prefix_select<T, K, K - 1>(acc, v, nv, scale);
 }
 
 template <typename T>
@@ -260,7 +301,7 @@ __device__ __forceinline__ void reduce_and_store(Acc<kGreedy>& acc, float* red, 
         a = v.v;
         b = __int_as_float(v.i);
     } else {
-        MS v = warp_merge_ms(acc.ms);
+        MS v = warp_merge_ms_maxfirst(acc.ms);
         a = v.m;
         b = v.s;
     }
@@ -305,19 +346,6 @@ __device__ __forceinline__ void fold_vector(Acc<kGreedy>& acc, const uint4& w, i
 // ============================================================================
 // TMA bulk-copy variant.
 
-// Ring geometry of the bulk-copy variant (compile-time; defaults tuned on B200).
-#ifndef SV_STAGE_BYTES
-#define SV_STAGE_BYTES 16384
-#endif
-#ifndef SV_TMA_CONSUMER_WARPS
-#define SV_TMA_CONSUMER_WARPS 16
-#endif
-#ifndef SV_TMA_STAGES
-#define SV_TMA_STAGES 8
-#endif
-#ifndef SV_TMA_CTAS_PER_SM
-#define SV_TMA_CTAS_PER_SM 1
-#endif
 constexpr int kStageBytes = SV_STAGE_BYTES;
 
 struct StageMeta {
@@ -433,7 +461,6 @@ row_stats_tma_kernel(const StatsParams p) {
     // the named barrier 1 stays in step even after a timeout; wait outcomes are
     // made warp-uniform with __all_sync before anyone acts on them.
     Acc<kGreedy> acc;
-    const uint64_t scale2 = pack2(p.scale, p.scale);
     uint32_t stage = 0;
     int parity_item = 0;
     for (int64_t item = blockIdx.x; item < total_items; item += gridDim.x, parity_item ^= 1) {
@@ -462,12 +489,19 @@ row_stats_tma_kernel(const StatsParams p) {
                 }
             } else {
                 uint4 vv[kVecPerThread];
+                if (nvec == kVecPerThread * kConsumers) {  // full stage: no guards
 #pragma unroll
-                for (int k = 0; k < kVecPerThread; ++k) {
-                    const int v = tid + k * kConsumers;
-                    vv[k] = v < nvec ? ld_shared_v4(buf + 16 * v) : neg_inf_vector<T>();
+                    for (int k = 0; k < kVecPerThread; ++k) vv[k] = ld_shared_v4(buf + 16 * (tid + k * kConsumers));
+                    fold_vectors<T, kVecPerThread>(acc, vv, p.scale);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < kVecPerThread; ++k) {
+                        const int v = tid + k * kConsumers;
+                        vv[k] = v < nvec ? ld_shared_v4(buf + 16 * v) : make_uint4(0, 0, 0, 0);
+                    }
+                    const int nv = nvec > tid ? (nvec - tid + kConsumers - 1) / kConsumers : 0;
+                    fold_vectors_count<T, kVecPerThread>(acc, vv, nv, p.scale);
                 }
-                fold_vectors<T, kVecPerThread>(acc, vv, p.scale, scale2);
             }
             __syncwarp();
             if ((tid & 31) == 0) mbar_arrive(empty + slot);
@@ -487,6 +521,8 @@ row_stats_tma_kernel(const StatsParams p) {
                                                  p.partials + partial_idx, failed);
     }
     named_barrier_sync(2, kThreads);
+    // this CTA is done: the dependent draw kernel may start its prologue here
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
 }
 
 // ============================================================================
@@ -496,42 +532,50 @@ template <typename T, bool kGreedy, bool kVec, int kThreads>
 __global__ void __launch_bounds__(kThreads)
 row_stats_ldg_kernel(const StatsParams p) {
     constexpr int kWarps = kThreads / 32;
-    constexpr int kUnroll = 4;
+    constexpr int kUnroll = SV_LDG_UNROLL;
     extern __shared__ __align__(16) int ldg_row_start[];
     __shared__ int scan_scratch[32];
     __shared__ float red[2][3 * kWarps];
     build_row_prefix<kThreads>(p, ldg_row_start, scan_scratch);
     const int64_t total_items = (int64_t)ldg_row_start[p.nB] * p.C;
     const int tid = threadIdx.x;
-    const uint64_t scale2 = pack2(p.scale, p.scale);
     int parity_item = 0;
     for (int64_t item = blockIdx.x; item < total_items; item += gridDim.x, parity_item ^= 1) {
         const ItemDesc d = decode_item<T>(p, ldg_row_start, item);
         Acc<kGreedy> acc;
         acc.reset();
         if constexpr (kVec) {
+            // Software-pipelined: the next batch of kUnroll vectors is in
+            // flight while the current one is folded.
             const int64_t bytes_all = int64_t(d.e1 - d.e0) * Logit<T>::kSize;
             const int nvec = static_cast<int>(bytes_all >> 4);
             const unsigned char* src = d.row + int64_t(d.e0) * Logit<T>::kSize;
-            for (int v0 = tid; v0 < nvec; v0 += kThreads * kUnroll) {
-                uint4 w[kUnroll];
+            constexpr int kStride = kThreads * kUnroll;
+            uint4 cur[kUnroll];
+#pragma unroll
+            for (int k = 0; k < kUnroll; ++k) {
+                const int v = tid + k * kThreads;
+                cur[k] = v < nvec ? ld_global_stream_v4(src + 16 * int64_t(v)) : neg_inf_vector<T>();
+            }
+            for (int v0 = tid; v0 < nvec; v0 += kStride) {
+                uint4 nxt[kUnroll];
 #pragma unroll
                 for (int k = 0; k < kUnroll; ++k) {
-                    const int v = v0 + k * kThreads;
-                    w[k] = v < nvec ? ld_global_stream_v4(src + 16 * int64_t(v)) : make_uint4(0, 0, 0, 0);
+                    const int v = v0 + kStride + k * kThreads;
+                    nxt[k] = v < nvec ? ld_global_stream_v4(src + 16 * int64_t(v)) : neg_inf_vector<T>();
                 }
                 if constexpr (kGreedy) {
 #pragma unroll
                     for (int k = 0; k < kUnroll; ++k) {
                         const int v = v0 + k * kThreads;
-                        if (v < nvec) fold_vector<T, true>(acc, w[k], d.e0 + v * Logit<T>::kPerVec, 0.f);
+                        if (v < nvec) fold_vector<T, true>(acc, cur[k], d.e0 + v * Logit<T>::kPerVec, 0.f);
                     }
                 } else {
-#pragma unroll
-                    for (int k = 0; k < kUnroll; ++k)
-                        if (v0 + k * kThreads >= nvec) w[k] = neg_inf_vector<T>();
-                    fold_vectors<T, kUnroll>(acc, w, p.scale, scale2);
+                    const int nv = (nvec - v0 + kThreads - 1) / kThreads;
+                    fold_vectors_count<T, kUnroll>(acc, cur, nv, p.scale);
                 }
+#pragma unroll
+                for (int k = 0; k < kUnroll; ++k) cur[k] = nxt[k];
             }
             const int tail0 = d.e0 + nvec * Logit<T>::kPerVec;
             if (tail0 + tid < d.e1) {
@@ -548,6 +592,8 @@ row_stats_ldg_kernel(const StatsParams p) {
         }
         reduce_and_store<kGreedy, kWarps>(acc, red[parity_item], 1, kThreads, p.partials + d.partial_idx, false);
     }
+    __syncthreads();
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
 }
 
 }  // namespace sv
