@@ -83,9 +83,34 @@ def parse_args():
 # workload bookkeeping
 
 
+def rank_seed(cfg: int, rank: int) -> int:
+    """Each rank verifies its own batch (weak scaling): rank r draws the
+    workload from seed config_seed(cfg) + 7919 * r."""
+    return config_seed(cfg) + 7919 * rank
+
+
 def make_rank_workload(cfg: int, rank: int):
     params = dict(CONFIGS[cfg])
-    return make_workload(seed=config_seed(cfg) + 7919 * rank, **params)
+    return make_workload(seed=rank_seed(cfg, rank), **params)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest of every rank's value (timing only; no data-path
+    collective).  Single process: the value itself."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(n_ranks: int, positions_per_step: int, steps: int, t_max_ms: float) -> float:
+    """Whole-job verified draft positions/s: every rank verified
+    positions_per_step positions per step; the job took the slowest rank's
+    time."""
+    return n_ranks * positions_per_step * steps / (t_max_ms / 1e3)
 
 
 def stats_pass_bytes(w, greedy=False) -> int:
@@ -379,13 +404,9 @@ def run_ours_impl(args):
     region_ms = g0.elapsed_time(g1)
     step_ms = [a.elapsed_time(b) for a, b in step_ev] if step_ev is not None else [region_ms / K]
     t_rank = sum(step_ms) if flush_buf is not None else region_ms
-    t_max = t_rank
-    if n > 1:
-        t = torch.tensor([t_rank], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = max_over_ranks(t_rank, dev)
     positions = w.positions
-    value = n * positions * K / (t_max / 1e3)
+    value = aggregate_value(n, positions, K, t_max)
     ms_per_step = t_max / K
 
     # parity spot check of the timed outputs (host side, cheap): accept lengths in range
@@ -424,13 +445,9 @@ def run_ours_impl(args):
             ev[i][1].record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in ev)
-        if n > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
         assert np.array_equal(h_out[0].numpy(), g_len), "host entry point disagrees with device entry point"
-        e2e = {"value": n * positions * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": aggregate_value(n, positions, args.e2e_steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": int(h_out[0].nbytes + h_out[1].nbytes),
                "steps": args.e2e_steps, "ms_per_step": e2e_ms / args.e2e_steps}
 
