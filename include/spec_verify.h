@@ -92,7 +92,8 @@ typedef enum {
     SV_OK = 0,
     SV_EINVAL = 1,
     SV_ECUDA = 2,
-    SV_EUNSUPPORTED = 3
+    SV_EUNSUPPORTED = 3,
+    SV_ESCRATCH = 4    /* spec_verify_static_scratch: problem larger than its fixed scratch area */
 } sv_status;
 
 /* Problem shape.  row_stride is in elements between consecutive rows
@@ -187,6 +188,43 @@ SV_API const char *spec_verify_status_string(sv_status status);
 
 /* SV_ABI_VERSION of the built library. */
 SV_API int32_t spec_verify_abi_version(void);
+
+/* Allocation-free form of spec_verify, for callers that cannot hand the
+ * library any device memory of its own: code running while a stream is being
+ * captured into a CUDA graph (allocating then breaks or invalidates the
+ * capture), plain C hosts or runtimes that have no device allocator at hand,
+ * and services that reserve all device memory up front and forbid ad-hoc
+ * allocations.  The pages describe nothing like it; it exists only for those
+ * callers.
+ *
+ * It runs exactly the kernels of spec_verify, but their scratch (the
+ * row-statistics partials, spec_verify_workspace_bytes(shape) bytes) lives in
+ * one fixed array of SV_STATIC_SCRATCH_BYTES bytes inside the library
+ * instead of a caller-provided workspace.  Every GPU that loads the library
+ * holds that array until the process exits.  Inputs and outputs are still the
+ * caller's device buffers, as for spec_verify.
+ *
+ * - Shapes whose workspace would exceed SV_STATIC_SCRATCH_BYTES are rejected
+ *   with SV_ESCRATCH before anything is enqueued; use spec_verify then.
+ * - The library calls no cudaMalloc / cudaFree or any allocating routine.  The
+ *   first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call on a device before capturing a stream.
+ * - All calls share the one array and it keeps the last call's contents (no
+ *   part of it needs to start at zero).  Calls whose work overlaps on the GPU
+ *   (different streams, or different host threads, without ordering between
+ *   them) race on it and give wrong results; order them on one stream.
+ */
+#define SV_STATIC_SCRATCH_BYTES (1u << 20)
+SV_API sv_status spec_verify_static_scratch(const sv_shape *shape,
+                                            const void *target_logits,
+                                            const void *draft_logits,
+                                            const int32_t *draft_tokens,
+                                            const int32_t *draft_lens,
+                                            const float *uniforms,
+                                            float temperature, int32_t greedy,
+                                            int32_t *out_accept_len,
+                                            int32_t *out_tokens, void *stream);
 
 #ifdef __cplusplus
 }

@@ -35,6 +35,7 @@ class Status(enum.IntEnum):
     EINVAL = 1
     ECUDA = 2
     EUNSUPPORTED = 3
+    ESCRATCH = 4
 
 
 class StatsKernel(enum.IntEnum):
@@ -77,6 +78,8 @@ _SIGNATURES = {
                                 _VP, _SZ, _VP]),
     "spec_verify_status_string": (ctypes.c_char_p, [_I32]),
     "spec_verify_abi_version": (_I32, []),
+    "spec_verify_static_scratch": (_I32, [ctypes.POINTER(_Shape), _VP, _VP, _VP, _VP, _VP, _F32, _I32, _VP, _VP,
+                                          _VP]),
 }
 
 

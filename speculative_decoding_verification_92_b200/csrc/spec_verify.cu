@@ -36,6 +36,28 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
+// Fixed scratch of spec_verify_static_scratch (see the header): one array per
+// device, holding the row-statistics partials.  Host code may only use the
+// device address looked up with cudaGetSymbolAddress, cached per device.
+static __device__ __align__(256) unsigned char g_static_scratch[SV_STATIC_SCRATCH_BYTES];
+void* g_static_scratch_addr[kMaxDevices];
+
+cudaError_t static_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_static_scratch_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);  // with device `dev` current
+        if (e != cudaSuccess) return e;
+        g_static_scratch_addr[dev] = p;
+    }
+    *out = g_static_scratch_addr[dev];
+    return cudaSuccess;
+}
+
 cudaError_t device_info(DeviceInfo** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -415,12 +437,26 @@ sv_status spec_verify_host(const sv_shape* shape, const void* h_target_logits, c
     return e == cudaSuccess ? SV_OK : SV_ECUDA;
 }
 
+sv_status spec_verify_static_scratch(const sv_shape* shape, const void* target_logits, const void* draft_logits,
+                                     const int32_t* draft_tokens, const int32_t* draft_lens, const float* uniforms,
+                                     float temperature, int32_t greedy, int32_t* out_accept_len,
+                                     int32_t* out_tokens, void* stream) {
+    sv_status why;
+    if (!sv::shape_ok(shape, &why)) return why;
+    if (sv::workspace_bytes_for(*shape, sv::make_plan(*shape)) > SV_STATIC_SCRATCH_BYTES) return SV_ESCRATCH;
+    void* scratch = nullptr;
+    if (sv::static_scratch_address(&scratch) != cudaSuccess) return SV_ECUDA;
+    return spec_verify_ex(shape, target_logits, draft_logits, draft_tokens, draft_lens, uniforms, temperature,
+                          greedy, out_accept_len, out_tokens, scratch, SV_STATIC_SCRATCH_BYTES, stream, nullptr);
+}
+
 const char* spec_verify_status_string(sv_status status) {
     switch (status) {
         case SV_OK: return "ok";
         case SV_EINVAL: return "invalid argument";
         case SV_ECUDA: return "CUDA error";
         case SV_EUNSUPPORTED: return "unsupported shape or dtype";
+        case SV_ESCRATCH: return "problem larger than the static scratch area (use spec_verify with a workspace)";
     }
     return "unknown status";
 }
