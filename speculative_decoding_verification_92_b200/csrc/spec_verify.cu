@@ -20,7 +20,7 @@ constexpr int kTmaConsumerWarps = SV_TMA_CONSUMER_WARPS;
 constexpr int kTmaStages = SV_TMA_STAGES;
 constexpr int kTmaCtasPerSm = SV_TMA_CTAS_PER_SM;
 constexpr int kLdgThreads = 256;
-// Draw-kernel grid: about SV_DRAW_WAVES waves of 2 CTAs per SM.
+// Draw-kernel grid: about SV_DRAW_WAVES waves of kDrawCtasPerSm CTAs per SM.
 #ifndef SV_DRAW_WAVES
 #define SV_DRAW_WAVES 1
 #endif
@@ -95,13 +95,15 @@ Plan make_plan(const sv_shape& s) {
     Plan p;
     p.es = s.dtype == SV_BF16 ? 2 : 4;
     p.stride = s.row_stride ? s.row_stride : s.V;
+    // A chunk is a whole number of bulk-copy stages, so the row-statistics
+    // ring moves full stages except at the end of each row: the fewest
+    // stages per chunk that keep C <= kMaxChunks.
     const int64_t row_bytes = int64_t(s.V) * p.es;
-    int c = static_cast<int>((row_bytes + 32767) / 32768);
-    c = c < 1 ? 1 : (c > kMaxChunks ? kMaxChunks : c);
-    int ce = (s.V + c - 1) / c;
-    ce = (ce + 7) & ~7;
-    p.CE = ce;
-    p.C = (s.V + ce - 1) / ce;
+    const int64_t span = int64_t(kMaxChunks) * kStageBytes;
+    int64_t spc = (row_bytes + span - 1) / span;
+    spc = spc < 1 ? 1 : spc;
+    p.CE = static_cast<int>(spc * (kStageBytes / p.es));
+    p.C = static_cast<int>((s.V + p.CE - 1) / p.CE);
     return p;
 }
 
@@ -170,9 +172,9 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
 template <typename T>
 cudaError_t launch_draw(const DrawParams& base, int B, cudaStream_t st) {
     // A request's cluster has C2 = ceil(C / R) CTAs; R is chosen so that the
-    // whole batch is about SV_DRAW_WAVES waves of CTAs (2 per SM).
+    // whole batch is about SV_DRAW_WAVES waves of CTAs.
     auto k = verify_draw_kernel<T>;
-    const size_t smem = draw_smem_bytes(base.C, base.k_max);
+    const size_t smem = draw_smem_bytes(base.k_max, base.fast_draw != 0);
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return e;
     for (int b0 = 0; b0 < B; b0 += 65535) {
@@ -274,10 +276,15 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     dp.greedy = greedy ? 1 : 0;
     dp.stats_only = a.stats_only ? 1 : 0;
     dp.rows_aligned = rows_aligned ? 1 : 0;
+    dp.fast_draw = (rows_aligned && !greedy && !a.stats_only && int64_t(plan.CE) * plan.es <= kMaxChunkBytesFast) ? 1 : 0;
     {
-        const int64_t target_ctas = int64_t(dev.sm_count) * 2 * SV_DRAW_WAVES;
+        // fewest chunks per CTA that fit the batch in about SV_DRAW_WAVES
+        // waves, then spread evenly: C2 = ceil(C / r) CTAs of ceil(C / C2) chunks
+        const int64_t target_ctas = int64_t(dev.sm_count) * kDrawCtasPerSm * SV_DRAW_WAVES;
         int64_t r = (int64_t(plan.C) * s.B + target_ctas - 1) / target_ctas;
-        dp.R = static_cast<int>(r < 1 ? 1 : (r > plan.C ? plan.C : r));
+        r = r < 1 ? 1 : (r > plan.C ? plan.C : r);
+        const int C2 = static_cast<int>((plan.C + r - 1) / r);
+        dp.R = (plan.C + C2 - 1) / C2;
     }
     e = launch_draw<T>(dp, s.B, a.stream);
     return e == cudaSuccess ? SV_OK : SV_ECUDA;
@@ -312,7 +319,7 @@ sv_status run(const Call& a) {
 
     DeviceInfo* dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return SV_ECUDA;
-    if (draw_smem_bytes(plan.C, s.k_max) + 4096 > size_t(dev->max_smem_optin)) return SV_EUNSUPPORTED;
+    if (draw_smem_bytes(s.k_max, true) + 16384 > size_t(dev->max_smem_optin)) return SV_EUNSUPPORTED;
 
     // Kernel choice: the bulk-copy and vector paths need every row start on a
     // 16-byte boundary.

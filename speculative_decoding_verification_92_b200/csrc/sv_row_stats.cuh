@@ -399,10 +399,12 @@ row_stats_tma_kernel(const StatsParams p) {
     if (tid >= kConsumers) {
         // ----------------------------- producer warp -----------------------------
         const int lane = tid - kConsumers;
-        uint32_t stage = 0;
-        uint32_t last_round[kStages];
+        int slot = 0;               // ring position of the next stage
+        uint32_t phase = 0;         // parity of the ring round in progress
+        bool wrapped = false;       // the ring has been filled once
+        uint32_t last_phase[kStages];
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) last_round[s] = 0xffffffffu;
+        for (int s = 0; s < kStages; ++s) last_phase[s] = 0xffffffffu;
         bool stop = false;
         for (int64_t item = blockIdx.x; item < total_items && !stop; item += gridDim.x) {
             const ItemDesc d = decode_item<T>(p, row_start, item);
@@ -411,12 +413,10 @@ row_stats_tma_kernel(const StatsParams p) {
             const int tail_n = static_cast<int>((bytes_all - tma_bytes) / Logit<T>::kSize);
             const int nsub = tma_bytes == 0 ? 1 : static_cast<int>((tma_bytes + kStageBytes - 1) / kStageBytes);
             const unsigned char* src0 = d.row + int64_t(d.e0) * Logit<T>::kSize;
-            for (int sub = 0; sub < nsub; ++sub, ++stage) {
-                const int slot = stage % kStages;
-                const uint32_t round = stage / kStages;
+            for (int sub = 0; sub < nsub; ++sub) {
                 if (lane == 0) {
                     bool ok = true;
-                    if (round > 0) ok = mbar_wait_bounded(empty + slot, (round - 1) & 1u, p.timeout_ns);
+                    if (wrapped) ok = mbar_wait_bounded(empty + slot, phase ^ 1u, p.timeout_ns);
                     if (!ok) *abort_flag = 1;
                     if (*abort_flag) {
                         stop = true;
@@ -432,7 +432,7 @@ row_stats_tma_kernel(const StatsParams p) {
                         m.tail_n = tail_n;
                         m.flags = (sub == 0 ? 1 : 0) | (sub == nsub - 1 ? 2 : 0);
                         meta[slot] = m;
-                        last_round[slot] = round;
+                        last_phase[slot] = phase;
                         if (n > 0) {
                             mbar_arrive_expect_tx(full + slot, static_cast<uint32_t>(n));
                             bulk_copy_g2s(stage_buf + size_t(slot) * kStageBytes, src0 + off,
@@ -444,6 +444,11 @@ row_stats_tma_kernel(const StatsParams p) {
                 }
                 stop = __shfl_sync(0xffffffffu, stop, 0);
                 if (stop) break;
+                if (++slot == kStages) {
+                    slot = 0;
+                    phase ^= 1u;
+                    wrapped = true;
+                }
             }
         }
         // Wait until the consumers are done, then (only after a timeout) make
@@ -451,7 +456,7 @@ row_stats_tma_kernel(const StatsParams p) {
         named_barrier_sync(2, kThreads);
         if (lane == 0 && *abort_flag) {
             for (int s = 0; s < kStages; ++s)
-                if (last_round[s] != 0xffffffffu) (void)mbar_wait_bounded(full + s, last_round[s] & 1u, p.timeout_ns);
+                if (last_phase[s] != 0xffffffffu) (void)mbar_wait_bounded(full + s, last_phase[s], p.timeout_ns);
         }
         return;
     }
@@ -461,16 +466,15 @@ row_stats_tma_kernel(const StatsParams p) {
     // the named barrier 1 stays in step even after a timeout; wait outcomes are
     // made warp-uniform with __all_sync before anyone acts on them.
     Acc<kGreedy> acc;
-    uint32_t stage = 0;
+    int slot = 0;          // ring position of the next stage
+    uint32_t phase = 0;    // parity of the ring round in progress
     int parity_item = 0;
     for (int64_t item = blockIdx.x; item < total_items; item += gridDim.x, parity_item ^= 1) {
         acc.reset();
         bool failed = __any_sync(0xffffffffu, *abort_flag != 0);  // warp-uniform
         int64_t partial_idx = -1;
         while (!failed) {
-            const int slot = stage % kStages;
-            const uint32_t round = stage / kStages;
-            bool ok = !*abort_flag && mbar_wait_bounded(full + slot, round & 1u, p.timeout_ns);
+            bool ok = !*abort_flag && mbar_wait_bounded(full + slot, phase, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 *abort_flag = 1;
@@ -505,7 +509,10 @@ row_stats_tma_kernel(const StatsParams p) {
             }
             __syncwarp();
             if ((tid & 31) == 0) mbar_arrive(empty + slot);
-            ++stage;
+            if (++slot == kStages) {
+                slot = 0;
+                phase ^= 1u;
+            }
             if (m.flags & 2) {
                 if (m.tail && tid < m.tail_n) {
                     const float z = Logit<T>::load(m.tail, tid);

@@ -44,6 +44,17 @@
 #include "spec_verify.h"
 #include "sv_common.cuh"
 
+// Draw-kernel geometry (compile time; defaults tuned on B200).
+#ifndef SV_DRAW_CTAS_PER_SM
+#define SV_DRAW_CTAS_PER_SM 2
+#endif
+#ifndef SV_DRAW_PIECE_VECS
+#define SV_DRAW_PIECE_VECS 512
+#endif
+#ifndef SV_DRAW_STAGES
+#define SV_DRAW_STAGES 4
+#endif
+
 namespace sv {
 
 namespace cg = cooperative_groups;
@@ -72,16 +83,36 @@ struct DrawParams {
     int32_t greedy;
     int32_t stats_only;
     int32_t rows_aligned;        // every row starts on a 16-byte boundary
+    int32_t fast_draw;           // ring-based draw pass (aligned rows, chunks of at most
+                                 // kMaxChunkBytesFast); the launch provides the ring
 };
 
 constexpr int kDrawThreads = 256;
 constexpr int kDrawWarps = kDrawThreads / 32;
+constexpr int kDrawCtasPerSm = SV_DRAW_CTAS_PER_SM;  // resident draw CTAs per SM the kernel is built for
 constexpr int kBatchVecs = 4;        // 16-byte vectors (per row) per thread in flight in the segment passes
 constexpr int kMaxDraftsPerThread = (SV_MAX_K + kDrawThreads - 1) / kDrawThreads;
 
-// Dynamic shared memory: partials[(2k+1) * C] float2 | lse_t[k+1] | lse_d[k] | p[k] | q[k]
-__host__ __device__ inline size_t draw_smem_bytes(int C, int k_max) {
-    return 8 * size_t(2 * k_max + 1) * size_t(C) + 4 * (size_t(k_max + 1) + 3 * size_t(k_max)) + 16;
+// Ring of the fast draw pass: kDrawStages stages, each holding kPieceVecs
+// 16-byte vectors of the target row and as many of the draft row.
+constexpr int kPieceVecs = SV_DRAW_PIECE_VECS;
+constexpr int kDrawStages = SV_DRAW_STAGES;
+constexpr int kPieceVecsPerThread = kPieceVecs / kDrawThreads;
+constexpr int kStageRowBytes = kPieceVecs * 16;
+static_assert(kPieceVecs % kDrawThreads == 0 && 1024 % kPieceVecs == 0, "a piece must divide a 16 KiB stage");
+constexpr size_t kDrawRingBytes = size_t(kDrawStages) * 2 * kStageRowBytes;
+constexpr int kSegVecs = 32;  // vectors per segment: one warp-wide 16-byte load
+// The fast path takes chunks of at most kMaxChunkBytesFast, i.e.
+// kMaxSegsPerChunk segments.
+constexpr int kMaxChunkBytesFast = 8 * 16384;
+constexpr int kMaxSegsPerChunk = kMaxChunkBytesFast / 16 / kSegVecs;
+
+// Dynamic shared memory: lse_t[k+1] | lse_d[k] | p[k] | q[k] | ring (fast draw only)
+__host__ __device__ inline size_t draw_scalar_bytes(int k_max) {
+    return (4 * (size_t(k_max + 1) + 3 * size_t(k_max)) + 127) & ~size_t(127);
+}
+__host__ __device__ inline size_t draw_smem_bytes(int k_max, bool ring) {
+    return draw_scalar_bytes(k_max) + (ring ? kDrawRingBytes : 0);
 }
 
 // Block-wide inclusive scan of one float per thread; returns the thread's
@@ -231,131 +262,241 @@ __device__ __noinline__ int segment_walk(const WeightRow& r, bool resid, int lo,
     return found >= 0 ? found : last;
 }
 
-constexpr int kWarpIters = 16;  // 32-vector iterations per warp run in the coalesced draw pass
-
-// Coalesced pass over the chunk [e0, e0+n) of row j: warp w owns vectors
-// [w*WV, (w+1)*WV) of the chunk (the last, partial vector at the row end is
-// read element-wise); vs[it] = weight sum of vector w*WV + 32*it + lane.
-// Returns this warp's total (same value in every lane).
+// Weights of the PV elements of one 16-byte vector (tz from the target row,
+// ty from the draft row), the element at row index zero_at (one-hot draw)
+// set to 0; returns their sum, added in element order.
 template <typename T, bool kResid>
-__device__ __forceinline__ float chunk_vector_sums(const WeightRow& r, int e0, int n, int WV,
-                                                   float (&vs)[kWarpIters]) {
-    constexpr int PV = Logit<T>::kPerVec;
-    constexpr int ES = Logit<T>::kSize;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nfull = n / PV;                 // complete vectors
-    const int nvec = (n + PV - 1) / PV;       // including a partial last one
-    constexpr int kBatch = kResid ? 4 : 8;  // iterations whose loads are in flight together
-    float tot = 0.f;
-#pragma unroll
-    for (int half = 0; half < kWarpIters; half += kBatch) {
-        if (half * 32 >= WV) {  // uniform: nothing left for any lane
-#pragma unroll
-            for (int k = 0; k < kBatch; ++k) vs[half + k] = 0.f;
-            continue;
-        }
-        uint4 a[kBatch], d[kBatch];
-#pragma unroll
-        for (int k = 0; k < kBatch; ++k) {
-            const int it = half + k;
-            const int v = warp * WV + it * 32 + lane;
-            if (it * 32 + lane < WV && v < nfull) {
-                a[k] = ld_global_stream_v4(r.trow + int64_t(e0 + v * PV) * ES);
-                if constexpr (kResid) d[k] = ld_global_stream_v4(r.drow + int64_t(e0 + v * PV) * ES);
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < kBatch; ++k) {
-            const int it = half + k;
-            const int v = warp * WV + it * 32 + lane;
-            float sum = 0.f;
-            if (it * 32 + lane < WV && v < nfull) {
-                float zf[PV], yf[PV];
-                Logit<T>::unpack(a[k], zf);
-                if constexpr (kResid) Logit<T>::unpack(d[k], yf);
-#pragma unroll
-                for (int i = 0; i < PV; ++i) {
-                    float w = draw_weight<kResid>(r, zf[i], kResid ? yf[i] : 0.f);
-                    if (!kResid && e0 + v * PV + i == r.zero_at) w = 0.f;
-                    sum += w;
-                }
-            } else if (it * 32 + lane < WV && v < nvec) {  // partial vector at the row end
-                for (int i = 0; v * PV + i < n; ++i) {
-                    const int idx = e0 + v * PV + i;
-                    float w = draw_weight<kResid>(r, Logit<T>::load(r.trow, idx),
-                                                  kResid ? Logit<T>::load(r.drow, idx) : 0.f);
-                    if (!kResid && idx == r.zero_at) w = 0.f;
-                    sum += w;
-                }
-            }
-            vs[it] = sum;
-            tot += sum;
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    return tot;
-}
-
-// Within one vector (row elements first .. first+count-1, count <= PV): the
-// first element with positive weight at which acc0 + running weight exceeds
-// target, else the last positive-weight element, else -1.  A full aligned
-// vector is read with one 16-byte load per row.
-template <typename T>
-__device__ __noinline__ int vector_walk(const WeightRow& r, bool resid, int first, int count, bool vec_ok,
-                                        float acc0, float target) {
+__device__ __forceinline__ float vector_weights(const WeightRow& r, const uint4& tz, const uint4& ty, int idx0,
+                                                float (&w)[Logit<T>::kPerVec]) {
     constexpr int PV = Logit<T>::kPerVec;
     float z[PV], y[PV];
-    if (vec_ok && count == PV) {
-        Logit<T>::unpack(ld_global_stream_v4(r.trow + int64_t(first) * Logit<T>::kSize), z);
-        if (resid) Logit<T>::unpack(ld_global_stream_v4(r.drow + int64_t(first) * Logit<T>::kSize), y);
-    } else {
-#pragma unroll
-        for (int i = 0; i < PV; ++i) {
-            z[i] = i < count ? Logit<T>::load(r.trow, first + i) : -INFINITY;
-            y[i] = (resid && i < count) ? Logit<T>::load(r.drow, first + i) : 0.f;
-        }
-    }
-    float acc = acc0;
-    int found = -1, last = -1;
+    Logit<T>::unpack(tz, z);
+    if constexpr (kResid) Logit<T>::unpack(ty, y);
+    float sum = 0.f;
 #pragma unroll
     for (int i = 0; i < PV; ++i) {
-        if (i >= count || found >= 0) continue;
-        const int idx = first + i;
-        const float w = resid ? draw_weight<true>(r, z[i], y[i])
-                              : (idx == r.zero_at ? 0.f : draw_weight<false>(r, z[i], 0.f));
-        if (w > 0.f) {
-            last = idx;
-            acc += w;
-            if (acc > target) found = idx;
+        float wi = draw_weight<kResid>(r, z[i], kResid ? y[i] : 0.f);
+        if (!kResid && idx0 + i == r.zero_at) wi = 0.f;
+        w[i] = wi;
+        sum += wi;
+    }
+    return sum;
+}
+
+// The same for the partial vector at the end of a row (count < PV
+// elements), read element-wise; absent elements get weight 0.
+template <typename T, bool kResid>
+__device__ __forceinline__ float tail_weights(const WeightRow& r, int idx0, int count,
+                                              float (&w)[Logit<T>::kPerVec]) {
+    constexpr int PV = Logit<T>::kPerVec;
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < PV; ++i) {
+        w[i] = 0.f;
+        if (i < count) {
+            const int idx = idx0 + i;
+            float wi = draw_weight<kResid>(r, Logit<T>::load(r.trow, idx), kResid ? Logit<T>::load(r.drow, idx) : 0.f);
+            if (!kResid && idx == r.zero_at) wi = 0.f;
+            w[i] = wi;
+            sum += wi;
         }
     }
-    return found >= 0 ? found : last;
+    return sum;
+}
+
+// Fast draw pass over the nch consecutive chunks k0 .. k0+nch-1 of row j
+// (and of the draft row j for the residual).  The chunks stream through a
+// ring of kDrawStages shared-memory stages filled by 16-byte cp.async copies
+// (every thread copies the vectors it will read, so no register holds data
+// in flight); the weight sum of each segment of kSegVecs vectors goes to
+// s_seg[(k - k0) * kMaxSegsPerChunk + segment].  Chunks are whole multiples
+// of 16 KiB, so every stage but the last of the row is full.
+template <typename T, bool kResid>
+__device__ __noinline__ void draw_pass(const WeightRow r, int k0, int nch, int CE, int V, unsigned char* ring,
+                                       float* s_seg) {
+    constexpr int PV = Logit<T>::kPerVec;
+    constexpr int ES = Logit<T>::kSize;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int spst = CE / PV / kPieceVecs;  // stages per full chunk
+    const int n_last = min(V - (k0 + nch - 1) * CE, CE);
+    const int G = (nch - 1) * spst + ((n_last + PV - 1) / PV + kPieceVecs - 1) / kPieceVecs;
+    auto issue = [&](int g) {
+        if (g < G) {
+            const int slot = g / spst, piece = g - slot * spst;
+            const int e0 = (k0 + slot) * CE;
+            const int nfull = min(V - e0, CE) / PV;
+            unsigned char* buf = ring + size_t(g % kDrawStages) * 2 * kStageRowBytes;
+#pragma unroll
+            for (int i = 0; i < kPieceVecsPerThread; ++i) {
+                const int lv = tid + i * kDrawThreads;  // vector within the piece
+                const int v = piece * kPieceVecs + lv;  // vector within the chunk
+                if (v < nfull) {
+                    cp_async_16(buf + lv * 16, r.trow + int64_t(e0 + v * PV) * ES);
+                    if constexpr (kResid) cp_async_16(buf + kStageRowBytes + lv * 16, r.drow + int64_t(e0 + v * PV) * ES);
+                }
+            }
+        }
+        cp_async_commit();  // possibly empty: keeps the group count per iteration fixed
+    };
+#pragma unroll
+    for (int g = 0; g < kDrawStages - 1; ++g) issue(g);
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+        issue(g + kDrawStages - 1);  // into the stage consumed in iteration g - 1
+        cp_async_wait<kDrawStages - 1>();
+        __syncthreads();             // every thread's copies of stage g have landed
+        const int slot = g / spst, piece = g - slot * spst;
+        const int e0 = (k0 + slot) * CE;
+        const int n = min(V - e0, CE);
+        const int nfull = n / PV, nvec = (n + PV - 1) / PV;
+        const unsigned char* buf = ring + size_t(g % kDrawStages) * 2 * kStageRowBytes;
+#pragma unroll
+        for (int i = 0; i < kPieceVecsPerThread; ++i) {
+            const int lv = tid + i * kDrawThreads;
+            const int v = piece * kPieceVecs + lv;
+            float w[Logit<T>::kPerVec];
+            float sum = 0.f;
+            if (v < nfull) {
+                const uint4 tz = ld_shared_v4(buf + lv * 16);
+                const uint4 ty = kResid ? ld_shared_v4(buf + kStageRowBytes + lv * 16) : tz;
+                sum = vector_weights<T, kResid>(r, tz, ty, e0 + v * PV, w);
+            } else if (v < nvec) {
+                sum = tail_weights<T, kResid>(r, e0 + v * PV, n - v * PV, w);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            // lane 0 holds the first vector of its warp's segment
+            if (lane == 0) s_seg[slot * kMaxSegsPerChunk + v / kSegVecs] = sum;
+        }
+        __syncthreads();             // stage g is free for reuse
+    }
+}
+
+// Inclusive warp scan of v over lanes.
+__device__ __forceinline__ float warp_scan_incl(float v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+
+// Final step of the fast draw, run by one warp: inside chunk [e0, e0+n)
+// whose segment sums are segs[0 .. nseg), find the element at which the
+// running weight first exceeds `target` -- segment (a scan over lanes, each
+// lane holding consecutive segments), then vector (one warp-wide re-read of
+// the segment, one vector per lane, and a scan over lanes), then element.
+// Rounding that leaves the target past every block takes the last block with
+// positive weight instead.  Returns the row index (same in every lane), or -1
+// when the chunk has no positive weight.
+template <typename T>
+__device__ __noinline__ int draw_select(const WeightRow r, bool resid, int e0, int n, const float* segs,
+                                        float target) {
+    constexpr int PV = Logit<T>::kPerVec;
+    constexpr int ES = Logit<T>::kSize;
+    const int lane = threadIdx.x & 31;
+    const int nfull = n / PV, nvec = (n + PV - 1) / PV;
+    const int nseg = (nvec + kSegVecs - 1) / kSegVecs;
+    // segment
+    const int cps = (nseg + 31) / 32;
+    const int s0 = lane * cps;
+    const int ns = min(cps, max(0, nseg - s0));
+    float mine = 0.f;
+    for (int i = 0; i < ns; ++i) mine += segs[s0 + i];
+    const float li = warp_scan_incl(mine);
+    unsigned cross = __ballot_sync(0xffffffffu, mine > 0.f && li > target);
+    unsigned pos = __ballot_sync(0xffffffffu, mine > 0.f);
+    int lsel = cross ? __ffs(cross) - 1 : (pos ? 31 - __clz(pos) : -1);
+    if (lsel < 0) return -1;
+    int seg = 0;
+    float t_seg = INFINITY;
+    if (lane == lsel) {
+        const float t1 = cross ? target : INFINITY;
+        float run = li - mine, before = 0.f, last_before = 0.f;
+        int isel = -1, ilast = -1;
+        for (int i = 0; i < ns; ++i) {
+            const float w = segs[s0 + i];
+            if (w > 0.f) {
+                ilast = i;
+                last_before = run;
+                if (run + w > t1) { isel = i; before = run; break; }
+            }
+            run += w;
+        }
+        const bool hit = isel >= 0;
+        if (!hit) { isel = ilast; before = last_before; }
+        seg = s0 + isel;
+        t_seg = hit ? t1 - before : INFINITY;
+    }
+    seg = __shfl_sync(0xffffffffu, seg, lsel);
+    t_seg = __shfl_sync(0xffffffffu, t_seg, lsel);
+    // vector: lane l re-reads vector seg * kSegVecs + l of the chunk
+    const int v = seg * kSegVecs + lane;
+    float w[PV];
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < PV; ++i) w[i] = 0.f;
+    if (v < nfull) {
+        const uint4 tz = ld_global_stream_v4(r.trow + int64_t(e0 + v * PV) * ES);
+        if (resid) {
+            const uint4 ty = ld_global_stream_v4(r.drow + int64_t(e0 + v * PV) * ES);
+            sum = vector_weights<T, true>(r, tz, ty, e0 + v * PV, w);
+        } else {
+            sum = vector_weights<T, false>(r, tz, tz, e0 + v * PV, w);
+        }
+    } else if (v < nvec) {
+        sum = resid ? tail_weights<T, true>(r, e0 + v * PV, n - v * PV, w)
+                    : tail_weights<T, false>(r, e0 + v * PV, n - v * PV, w);
+    }
+    const float lv = warp_scan_incl(sum);
+    cross = __ballot_sync(0xffffffffu, sum > 0.f && lv > t_seg);
+    pos = __ballot_sync(0xffffffffu, sum > 0.f);
+    lsel = cross ? __ffs(cross) - 1 : (pos ? 31 - __clz(pos) : -1);
+    if (lsel < 0) return -1;
+    // element, in the selected lane's registers
+    int found = -1, last = -1;
+    if (lane == lsel) {
+        const float t2 = cross ? t_seg : INFINITY;
+        float run = lv - sum;
+#pragma unroll
+        for (int i = 0; i < PV; ++i) {
+            if (w[i] > 0.f && found < 0) {
+                last = i;
+                run += w[i];
+                if (run > t2) found = i;
+            }
+        }
+        found = e0 + v * PV + (found >= 0 ? found : last);
+    }
+    return __shfl_sync(0xffffffffu, found, lsel);
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kDrawThreads, 2)
+__global__ void __launch_bounds__(kDrawThreads, kDrawCtasPerSm)
 verify_draw_kernel(const DrawParams p) {
-    extern __shared__ __align__(16) unsigned char draw_dsm[];
+    extern __shared__ __align__(128) unsigned char draw_dsm[];
     __shared__ float s_Wc[kMaxChunks];
     __shared__ float s_warp[kDrawWarps];
     __shared__ float s_incl[kDrawThreads];
-    __shared__ int s_first, s_fail, s_cstar, s_mode, s_found, s_seg, s_lastseg;
+    __shared__ float s_seg[kMaxChunks * kMaxSegsPerChunk];  // segment sums of the fast draw pass
+    __shared__ int s_first, s_fail, s_cstar, s_mode, s_found, s_segsel, s_lastseg;
     __shared__ float s_local_target;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int c = blockIdx.x;
     const int b = p.b0 + blockIdx.y;
     const int K = p.k_max;
-    const int R = 2 * K + 1;
+    const int nslots = 2 * K + 1;  // partial rows per request
     const int C = p.C;
     const int64_t esz = Logit<T>::kSize;
-    float2* s_part = reinterpret_cast<float2*>(draw_dsm);   // used rows, compact: row r at r*C
-    float* s_lse_t = reinterpret_cast<float*>(s_part + size_t(R) * C);
+    float* s_lse_t = reinterpret_cast<float*>(draw_dsm);
     float* s_lse_d = s_lse_t + (K + 1);
     float* s_p = s_lse_d + K;   // gathered z(x_i), then p_i
     float* s_q = s_p + K;       // gathered y(x_i), then q_i
     int* s_arg_t = reinterpret_cast<int*>(s_lse_t);  // greedy: argmax per target row
+    unsigned char* ring = draw_dsm + draw_scalar_bytes(K);
     const int32_t* x = p.tokens + int64_t(b) * K;
     int32_t* out_tok = p.out_tokens ? p.out_tokens + int64_t(b) * (K + 1) : nullptr;
     const bool has_draft = p.draft != nullptr && !p.greedy;
@@ -408,7 +549,8 @@ verify_draw_kernel(const DrawParams p) {
     }
 
     // 2. the row-statistics kernel's partials (this kernel is a programmatic
-    // dependent of it: wait for its completion before reading them) --------------
+    // dependent of it: wait for its completion before reading them), merged
+    // straight from global memory: G lanes per row, 32/G rows per warp at once
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (!ok) {
         write_failed(-1);
@@ -418,21 +560,15 @@ verify_draw_kernel(const DrawParams p) {
     const int n_t = L + 1;
     const int n_d = has_draft ? L : 0;
     const int nrows = n_t + n_d;
-    for (int idx = tid; idx < nrows * C; idx += kDrawThreads) {
-        const int row = idx / C, cc = idx - row * C;
-        const int slot = row < n_t ? row : K + 1 + (row - n_t);
-        s_part[idx] = p.partials[(int64_t(b) * R + slot) * C + cc];
-    }
-    __syncthreads();
-
-    // 3. merge the partials: G lanes per row, 32/G rows per warp at once -----------
     {
         const int G = C <= 1 ? 1 : (C <= 2 ? 2 : (C <= 4 ? 4 : 8));
         const int sub = lane / G, gl = lane - sub * G;
+        const float2* part_b = p.partials + int64_t(b) * nslots * C;
         for (int r0 = warp * (32 / G); r0 < nrows; r0 += kDrawWarps * (32 / G)) {
             const int row = r0 + sub;
             const bool act = row < nrows && gl < C;
-            const float2 v = act ? s_part[row * C + gl] : make_float2(-INFINITY, 0.f);
+            const int slot = row < n_t ? row : K + 1 + (row - n_t);
+            const float2 v = act ? part_b[int64_t(slot) * C + gl] : make_float2(-INFINITY, 0.f);
             bool bad;
             if (p.greedy) {
                 const int idx = act ? __float_as_int(v.y) : 0x7fffffff;
@@ -461,7 +597,7 @@ verify_draw_kernel(const DrawParams p) {
         return;
     }
 
-    // 4. p, q at the drafted ids; acceptance scan ----------------------------------
+    // 3. p, q at the drafted ids; acceptance scan ----------------------------------
 #pragma unroll
     for (int k = 0; k < kMaxDraftsPerThread; ++k) {
         const int i = tid + k * kDrawThreads;
@@ -507,42 +643,30 @@ verify_draw_kernel(const DrawParams p) {
     }
     if (p.greedy) return;
 
-    // 5. final draw on row j: chunk weights and the chunk that holds u*W ---------------
+    // 4. final draw on row j: chunk weights and the chunk that holds u*W ---------------
     WeightRow wr;
     wr.trow = trow_of(j);
     wr.drow = (has_draft && j < L) ? drow_of(j) : nullptr;
     wr.scale = p.scale;
     wr.lse_p = s_lse_t[j];
     wr.lse_q = (has_draft && j < L) ? s_lse_d[j] : 0.f;
+    wr.zero_at = -1;
     const float ustar = __ldg(u + K);
     const bool vec_ok = p.rows_aligned != 0;
-    int mode = j == L ? kBonus : (has_draft ? kResidual : kOneHot);
-    constexpr int PV = Logit<T>::kPerVec;
-    const int WV_full = ((p.CE + PV - 1) / PV + kDrawWarps - 1) / kDrawWarps;  // vectors per warp run
-    const bool fast = vec_ok && WV_full <= 32 * kWarpIters;
+    const bool fast = p.fast_draw != 0;
+    const int mode = j == L ? kBonus : (has_draft ? kResidual : kOneHot);
     const int k_lo = c * p.R, k_hi = min(C, k_lo + p.R);  // this CTA's chunks
-    float vs[kWarpIters];
-    float wtot = 0.f;          // this warp's total of the last chunk summed (fast path)
+    const float2* part_j = p.partials + (int64_t(b) * nslots + j) * C;  // row j's chunk partials
     float ssum = 0.f, excl = 0.f, incl = 0.f;
     auto chunk_bounds = [&](int k, int* e0, int* n) {
         *e0 = k * p.CE;
         *n = min(p.V - *e0, p.CE);
     };
-    // Sum of the draw weights over chunk k (block-wide; all threads get it).
-    auto chunk_total = [&](int k, bool resid) {
+    // Slow path: sum of the draw weights over chunk k from contiguous
+    // per-thread segments (block-wide; all threads get it).
+    auto chunk_total_slow = [&](int k, bool resid) {
         int e0, n;
         chunk_bounds(k, &e0, &n);
-        if (fast) {
-            const int WV = ((n + PV - 1) / PV + kDrawWarps - 1) / kDrawWarps;
-            wtot = resid ? chunk_vector_sums<T, true>(wr, e0, n, WV, vs) : chunk_vector_sums<T, false>(wr, e0, n, WV, vs);
-            __syncthreads();  // previous readers of s_warp are done
-            if (lane == 0) s_warp[warp] = wtot;
-            __syncthreads();
-            float t = 0.f;
-#pragma unroll
-            for (int w = 0; w < kDrawWarps; ++w) t += s_warp[w];
-            return t;
-        }
         int lo, hi;
         thread_segment<T>(e0, n, &lo, &hi);
         ssum = segment_sum<T>(wr, resid, lo, hi, vec_ok);
@@ -550,157 +674,111 @@ verify_draw_kernel(const DrawParams p) {
         return s_incl[kDrawThreads - 1];
     };
 
+    bool have_segs = false;  // s_seg holds this CTA's chunks for the residual weights
     if (mode == kResidual) {
         // every CTA sums its chunks; the sums are exchanged across the cluster
-        wr.zero_at = -1;
         cg::cluster_group cluster = cg::this_cluster();
         const int C2 = (C + p.R - 1) / p.R;
-        for (int k = k_lo; k < k_hi; ++k) {
-            const float Wk = chunk_total(k, true);
-            if (tid < C2) {
-                float* remote = cluster.map_shared_rank(&s_Wc[0], tid);
-                remote[k] = Wk;
+        if (fast) {
+            draw_pass<T, true>(wr, k_lo, k_hi - k_lo, p.CE, p.V, ring, s_seg);
+            have_segs = true;
+            if (warp < k_hi - k_lo) {  // warp w totals chunk k_lo + w (R <= 8 warps)
+                int e0, n;
+                chunk_bounds(k_lo + warp, &e0, &n);
+                const int nseg = ((n + Logit<T>::kPerVec - 1) / Logit<T>::kPerVec + kSegVecs - 1) / kSegVecs;
+                float t = 0.f;
+                for (int s = lane; s < nseg; s += 32) t += s_seg[warp * kMaxSegsPerChunk + s];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+                if (lane < C2) cluster.map_shared_rank(&s_Wc[0], lane)[k_lo + warp] = t;
+            }
+        } else {
+            for (int k = k_lo; k < k_hi; ++k) {
+                const float Wk = chunk_total_slow(k, true);
+                if (tid < C2) cluster.map_shared_rank(&s_Wc[0], tid)[k] = Wk;
             }
         }
         cluster.sync();
     }
 
-    if (tid == 0) {
-        float W[kMaxChunks];
-        float total = 0.f;
-        for (int cc = 0; cc < C; ++cc) {
+    if (warp == 0) {
+        // lane cc holds chunk cc's weight
+        float W = 0.f;
+        int m2 = mode;
+        if (lane < C) {
             if (mode == kResidual) {
-                W[cc] = s_Wc[cc];
+                W = s_Wc[lane];
             } else {
-                const float2 pp = s_part[j * C + cc];
-                W[cc] = pp.y * exp2f(pp.x - wr.lse_p);
+                const float2 pp = part_j[lane];
+                W = pp.y * exp2f(pp.x - wr.lse_p);
+                if (mode == kOneHot && lane == __ldg(x + j) / p.CE) W = fmaxf(0.f, W - s_p[j]);
             }
         }
-        if (mode == kOneHot) {
-            const int cx = __ldg(x + j) / p.CE;
-            W[cx] = fmaxf(0.f, W[cx] - s_p[j]);
-        }
-        for (int cc = 0; cc < C; ++cc) total += W[cc];
+        float total = W;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
         if (!(total > 0.f)) {
             // zero residual mass (p == q numerically): draw from p_j
-            mode = kBonus;
-            total = 0.f;
-            for (int cc = 0; cc < C; ++cc) {
-                const float2 pp = s_part[j * C + cc];
-                W[cc] = pp.y * exp2f(pp.x - wr.lse_p);
-                total += W[cc];
+            m2 = kBonus;
+            W = 0.f;
+            if (lane < C) {
+                const float2 pp = part_j[lane];
+                W = pp.y * exp2f(pp.x - wr.lse_p);
             }
+            total = W;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
         }
         const float target = ustar * total;
-        int cstar = -1, last_pos = 0;
-        float before = 0.f, run = 0.f;
-        for (int cc = 0; cc < C; ++cc) {
-            if (W[cc] > 0.f) last_pos = cc;
-            if (cstar < 0 && run + W[cc] > target) { cstar = cc; before = run; }
-            run += W[cc];
+        const float wi = warp_scan_incl(W);
+        const unsigned cross = __ballot_sync(0xffffffffu, W > 0.f && wi > target);
+        const unsigned pos = __ballot_sync(0xffffffffu, W > 0.f);
+        const int cstar = cross ? __ffs(cross) - 1 : (pos ? 31 - __clz(pos) : 0);
+        const float before = __shfl_sync(0xffffffffu, wi - W, cstar);
+        if (lane == 0) {
+            s_cstar = cstar;
+            s_mode = m2;
+            s_local_target = cross ? fmaxf(0.f, target - before) : INFINITY;
+            s_found = -1;
+            s_segsel = 0x7fffffff;
+            s_lastseg = -1;
         }
-        if (cstar < 0) {
-            cstar = last_pos;
-            before = 0.f;
-            for (int cc = 0; cc < cstar; ++cc) before += W[cc];
-        }
-        s_cstar = cstar;
-        s_mode = mode;
-        s_local_target = fmaxf(0.f, target - before);
-        s_found = -1;
-        s_seg = 0x7fffffff;
-        s_lastseg = -1;
     }
     __syncthreads();
     const int kstar = s_cstar;
     if (kstar < k_lo || kstar >= k_hi) return;
 
-    // 6. inverse CDF inside chunk k* ---------------------------------------------------
+    // 5. inverse CDF inside chunk k* ---------------------------------------------------
     const bool resid = s_mode == kResidual;
-    // the residual pass already left chunk k*'s sums in registers when it was
-    // this CTA's only (hence last) chunk
-    const bool recompute = mode != s_mode || !resid || k_hi - k_lo != 1;
     const float target = s_local_target;
     wr.zero_at = s_mode == kOneHot ? __ldg(x + j) : -1;
     int e0, n;
     chunk_bounds(kstar, &e0, &n);
-    if (recompute) (void)chunk_total(kstar, resid);
     if (fast) {
-        const int WV = ((n + PV - 1) / PV + kDrawWarps - 1) / kDrawWarps;
-        __syncthreads();
-        if (tid == 0) {
-            // warp whose run holds the target (first with positive total), or
-            // the last positive warp when rounding leaves the target past it
-            float run = 0.f;
-            int ws = -1, wl = -1;
-            float wb = 0.f;
-            for (int w = 0; w < kDrawWarps; ++w) {
-                const float t = s_warp[w];
-                if (t > 0.f) {
-                    wl = w;
-                    if (ws < 0 && run + t > target) { ws = w; wb = run; }
-                }
-                run += t;
-            }
-            s_seg = ws >= 0 ? ws : wl;
-            s_incl[0] = ws >= 0 ? target - wb : INFINITY;
+        const float* segs = s_seg + (kstar - k_lo) * kMaxSegsPerChunk;
+        if (!(resid && have_segs)) {
+            // bonus or one-hot draw: one pass over chunk k* alone
+            draw_pass<T, false>(wr, kstar, 1, p.CE, p.V, ring, s_seg);
+            segs = s_seg;
         }
-        __syncthreads();
-        if (warp == s_seg) {
-            const float t1 = s_incl[0];
-            // iteration holding the target within this warp's run
-            float run = 0.f;
-            int its = -1, itl = -1;
-            float itb = 0.f;
-#pragma unroll
-            for (int it = 0; it < kWarpIters; ++it) {
-                float tsum = vs[it];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, o);
-                if (tsum > 0.f) {
-                    itl = it;
-                    if (its < 0 && run + tsum > t1) { its = it; itb = run; }
-                }
-                run += tsum;
-            }
-            const int it_sel = its >= 0 ? its : itl;
-            const float t2 = its >= 0 ? t1 - itb : INFINITY;
-            float mine = 0.f;
-#pragma unroll
-            for (int it = 0; it < kWarpIters; ++it)
-                if (it == it_sel) mine = vs[it];
-            // lane holding the target: inclusive scan over lanes
-            float li = mine;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, li, o);
-                if (lane >= o) li += v;
-            }
-            const unsigned cross = __ballot_sync(0xffffffffu, mine > 0.f && li > t2);
-            const unsigned pos = __ballot_sync(0xffffffffu, mine > 0.f);
-            const int lsel = cross ? __ffs(cross) - 1 : (pos ? 31 - __clz(pos) : -1);
-            if (lsel >= 0 && lane == lsel) {
-                const int v = warp * WV + it_sel * 32 + lane;
-                const int first = e0 + v * PV;
-                const int count = min(PV, e0 + n - first);
-                s_found = vector_walk<T>(wr, resid, first, count, vec_ok, li - mine, cross ? t2 : INFINITY);
-            }
+        if (warp == 0) {
+            const int t = draw_select<T>(wr, resid, e0, n, segs, target);
+            if (lane == 0) out_tok[j] = t >= 0 ? t : e0;
         }
-        __syncthreads();
-        if (tid == 0) out_tok[j] = s_found >= 0 ? s_found : e0;
         return;
     }
 
     // slow path: contiguous per-thread segments, one block scan, one walk
+    (void)chunk_total_slow(kstar, resid);
     int lo, hi;
     thread_segment<T>(e0, n, &lo, &hi);
     if (ssum > 0.f) {
-        if (incl > target) atomicMin(&s_seg, tid);
+        if (incl > target) atomicMin(&s_segsel, tid);
         atomicMax(&s_lastseg, tid);
     }
     __syncthreads();
-    if (tid == s_seg) s_found = segment_walk<T>(wr, resid, lo, hi, vec_ok, excl, target);
-    else if (s_seg == 0x7fffffff && tid == s_lastseg)  // rounding left u*W past the last step
+    if (tid == s_segsel) s_found = segment_walk<T>(wr, resid, lo, hi, vec_ok, excl, target);
+    else if (s_segsel == 0x7fffffff && tid == s_lastseg)  // rounding left u*W past the last step
         s_found = segment_walk<T>(wr, resid, lo, hi, vec_ok, 0.f, INFINITY);
     __syncthreads();
     if (tid == 0) out_tok[j] = s_found >= 0 ? s_found : e0;

@@ -39,10 +39,13 @@ def test_status_strings():
     assert lib.spec_verify_status_string(99) == b"unknown status"
 
 
+STAGE_BYTES, MAX_CHUNKS = 16384, 8
+
+
 def plan_chunks(V, es):
-    c = max(1, min(8, -(-V * es // 32768)))
-    ce = -(-V // c)
-    ce = (ce + 7) & ~7
+    """Chunks are whole 16 KiB stages, as few per chunk as keep C <= 8."""
+    spc = max(1, -(-V * es // (MAX_CHUNKS * STAGE_BYTES)))
+    ce = spc * STAGE_BYTES // es
     return -(-V // ce), ce
 
 

@@ -114,7 +114,7 @@ def test_extreme_uniforms(u):
 def test_greedy_ties_across_chunk_boundary():
     V = 151936
     w = make_workload(B=3, k_max=2, V=V, dtype=BF16, seed=14, draft_mode="ids")
-    CE = 18992  # chunk length for this vocabulary
+    CE = 24576  # chunk length for this vocabulary: 3 stages of 16 KiB
     for b in range(3):
         for i in range(3):
             row = np.zeros(V, np.float32)

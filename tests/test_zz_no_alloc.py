@@ -43,7 +43,7 @@ def call_static(w, d, greedy=False):
 
 
 def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
-    w1 = make_config(2)                                   # 64 x 17 rows x 8 chunks of partials
+    w1 = make_config(2)                                   # 64 x 17 rows x 7 chunks of partials
     w2 = make_workload(B=33, k_max=12, V=20000, dtype="f32", seed=5, boost=4.0, draft_noise=0.3,
                        lens_choices=(0, 4, 12), lens_probs=(0.4, 0.3, 0.3))
     assert sv.workspace_bytes(w1.B, w1.k_max, w1.V, sv.BF16) <= SCRATCH_BYTES
