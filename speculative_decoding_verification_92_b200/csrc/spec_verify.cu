@@ -22,7 +22,7 @@ constexpr int kTmaCtasPerSm = SV_TMA_CTAS_PER_SM;
 constexpr int kLdgThreads = 256;
 // Draw-kernel grid: about SV_DRAW_WAVES waves of kDrawCtasPerSm CTAs per SM.
 #ifndef SV_DRAW_WAVES
-#define SV_DRAW_WAVES 1
+#define SV_DRAW_WAVES 2
 #endif
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;

@@ -46,13 +46,13 @@
 
 // Draw-kernel geometry (compile time; defaults tuned on B200).
 #ifndef SV_DRAW_CTAS_PER_SM
-#define SV_DRAW_CTAS_PER_SM 2
+#define SV_DRAW_CTAS_PER_SM 3
 #endif
 #ifndef SV_DRAW_PIECE_VECS
 #define SV_DRAW_PIECE_VECS 512
 #endif
 #ifndef SV_DRAW_STAGES
-#define SV_DRAW_STAGES 4
+#define SV_DRAW_STAGES 3
 #endif
 
 namespace sv {
