@@ -89,8 +89,9 @@ struct Plan {
     int64_t stride = 0;
 };
 
-// Rows are cut into at most kMaxChunks chunks of about 32 KiB; a chunk starts
-// on a 16-byte boundary of an aligned row.
+// Rows are cut into at most kMaxChunks chunks, each a whole number of the
+// row-statistics kernel's bulk-copy stages; a chunk starts on a 16-byte
+// boundary of an aligned row.
 Plan make_plan(const sv_shape& s) {
     Plan p;
     p.es = s.dtype == SV_BF16 ? 2 : 4;

@@ -308,9 +308,10 @@ __device__ __forceinline__ float tail_weights(const WeightRow& r, int idx0, int 
 // (and of the draft row j for the residual).  The chunks stream through a
 // ring of kDrawStages shared-memory stages filled by 16-byte cp.async copies
 // (every thread copies the vectors it will read, so no register holds data
-// in flight); the weight sum of each segment of kSegVecs vectors goes to
-// s_seg[(k - k0) * kMaxSegsPerChunk + segment].  Chunks are whole multiples
-// of 16 KiB, so every stage but the last of the row is full.
+// in flight and no barrier is needed); the weight sum of each segment of
+// kSegVecs vectors goes to s_seg[(k - k0) * kMaxSegsPerChunk + segment].
+// Chunks are whole multiples of 16 KiB, so every stage but the last of the
+// row is full.
 template <typename T, bool kResid>
 __device__ __noinline__ void draw_pass(const WeightRow r, int k0, int nch, int CE, int V, unsigned char* ring,
                                        float* s_seg) {
@@ -342,9 +343,13 @@ __device__ __noinline__ void draw_pass(const WeightRow r, int k0, int nch, int C
     for (int g = 0; g < kDrawStages - 1; ++g) issue(g);
 #pragma unroll 1
     for (int g = 0; g < G; ++g) {
-        issue(g + kDrawStages - 1);  // into the stage consumed in iteration g - 1
+        // Each thread copies exactly the vectors it reads back (vector
+        // tid + i * kDrawThreads of every piece), so its own wait_group makes
+        // stage g visible to it, and program order keeps the refill below of
+        // the stage it consumed in iteration g - 1 behind its reads: the
+        // ring needs no block barrier.
+        issue(g + kDrawStages - 1);
         cp_async_wait<kDrawStages - 1>();
-        __syncthreads();             // every thread's copies of stage g have landed
         const int slot = g / spst, piece = g - slot * spst;
         const int e0 = (k0 + slot) * CE;
         const int n = min(V - e0, CE);
@@ -368,8 +373,8 @@ __device__ __noinline__ void draw_pass(const WeightRow r, int k0, int nch, int C
             // lane 0 holds the first vector of its warp's segment
             if (lane == 0) s_seg[slot * kMaxSegsPerChunk + v / kSegVecs] = sum;
         }
-        __syncthreads();             // stage g is free for reuse
     }
+    __syncthreads();  // s_seg complete
 }
 
 // Inclusive warp scan of v over lanes.
