@@ -162,6 +162,43 @@ SV_API sv_status spec_verify_stats(const sv_shape *shape, const void *target_log
                             size_t workspace_bytes, void *stream,
                             const sv_options *opts);
 
+/* Acceptance simulation over a batch of drafted sequences, for training-time
+ * use: the same row-statistics pass and acceptance rule as spec_verify,
+ * without the final draw ("今热点：让AI草稿模型学会"照镜子"：训练时就知道自己会不会被
+ * 打回", sections "VAT怎么把"验收规则"塞进训练里" and "第二件事，改权重分配的锚点":
+ * the verification is simulated with the probability-ratio rule, everything
+ * from the first rejection on is marked rejected, and the per-position loss
+ * weights keep full weight up to the first rejection and start the decay
+ * curve there).  Inputs are those of spec_verify; uniforms may be NULL.
+ *
+ *   out_accept_prob [B][k_max]  a_i = min(1, p_i(x_i) / q_i(x_i)) for i < L_b,
+ *                               NaN for i >= L_b (q = 1 without draft logits);
+ *   out_expected_len [B]        E[j] = sum_{m=1..L_b} prod_{l<m} a_l, the
+ *                               expected number of accepted drafts;
+ *   out_first_reject [B]        (needs uniforms, else must be NULL) the first
+ *                               i < L_b with !(u_i < a_i), else L_b -- the j
+ *                               spec_verify returns for the same inputs;
+ *   out_weights [B][k_max]      (needs uniforms, else must be NULL) 1 for
+ *                               i <= j, decay^(i - j) for j < i < L_b, 0 for
+ *                               i >= L_b; decay in [0, 1] (0.8 is the fixed
+ *                               per-position curve of the EAGLE-3 recipe the
+ *                               page cites, 0 the hard cut-off of its
+ *                               ablation).
+ *
+ * out_accept_prob and out_expected_len are required.  A request with an
+ * invalid length or drafted id gets out_first_reject = -1 and NaN elsewhere;
+ * one whose statistics were lost to a wait timeout gets -2.  Same ownership,
+ * stream and workspace rules as spec_verify_stats. */
+SV_API sv_status spec_verify_accept_sim(const sv_shape *shape, const void *target_logits,
+                                        const void *draft_logits,
+                                        const int32_t *draft_tokens,
+                                        const int32_t *draft_lens, const float *uniforms,
+                                        float temperature, float decay,
+                                        float *out_accept_prob, float *out_expected_len,
+                                        int32_t *out_first_reject, float *out_weights,
+                                        void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
 /* Bytes of caller-provided device staging memory spec_verify_host needs. */
 SV_API size_t spec_verify_host_staging_bytes(const sv_shape *shape, int32_t has_draft,
                                       int32_t has_lens);

@@ -65,6 +65,10 @@ class Oracle:
                       dbl, i32, vp, vp, vp, vp, vp, vp, vp]
         f.restype = ctypes.c_int
         self._f = f
+        g = self._lib.oracle_accept_sim
+        g.argtypes = [i64, i32, i64, vp, vp, vp, vp, vp, dbl, vp, vp, vp, vp]
+        g.restype = ctypes.c_int
+        self._g = g
 
     def verify(self, target, draft, tokens, lens, uniforms, temperature=1.0,
                greedy=False, *, V=None, B=None, diag=False):
@@ -128,6 +132,32 @@ class Oracle:
         return out
 
 
+    def accept_sim(self, p, q, tokens, lens, uniforms=None, decay=0.8, *, V):
+        """Acceptance simulation from per-position probabilities ``p``, ``q``
+        [B, k_max] (float64, e.g. ``verify(..., diag=True)``'s): returns
+        ``a`` [B, k_max], ``e`` [B] and, with uniforms, ``j`` [B] and ``w``
+        [B, k_max] (else None)."""
+        p = np.ascontiguousarray(p, dtype=np.float64)
+        q = np.ascontiguousarray(q, dtype=np.float64)
+        B, k_max = p.shape
+        tokens = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, k_max)
+        if lens is not None:
+            lens = np.ascontiguousarray(lens, dtype=np.int32).reshape(B)
+        if uniforms is not None:
+            uniforms = np.ascontiguousarray(uniforms, dtype=np.float64).reshape(B, k_max + 1)
+        a = np.empty((B, k_max), np.float64)
+        e = np.empty(B, np.float64)
+        j = np.empty(B, np.int32) if uniforms is not None else None
+        w = np.empty((B, k_max), np.float64) if uniforms is not None else None
+
+        def ptr(x):
+            return None if x is None else x.ctypes.data
+
+        self._g(B, k_max, int(V), ptr(tokens), ptr(lens), ptr(p), ptr(q), ptr(uniforms), float(decay),
+                ptr(a), ptr(e), ptr(j), ptr(w))
+        return {"a": a, "e": e, "j": j, "w": w}
+
+
 _default: Oracle | None = None
 
 
@@ -141,3 +171,7 @@ def default() -> Oracle:
 
 def verify(*args, **kwargs):
     return default().verify(*args, **kwargs)
+
+
+def accept_sim(*args, **kwargs):
+    return default().accept_sim(*args, **kwargs)

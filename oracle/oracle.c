@@ -30,6 +30,14 @@
  *  [VAT-SEQ] "今热点：让AI草稿模型学会"照镜子"：训练时就知道自己会不会被打回"
  *            (001ce.com), section "先搞懂投机解码在干什么": verification runs in
  *            order and every draft after the first rejection is discarded.
+ *  [VAT-SIM] same page, section "VAT怎么把"验收规则"塞进训练里": training simulates
+ *            the verification with the same probability-ratio rule, and every
+ *            position from the first rejection on is labelled rejected.
+ *  [VAT-W]   same page, section "第二件事，改权重分配的锚点": per-position loss
+ *            weights keep full weight before the first rejection and start the
+ *            fixed decay curve (EAGLE-3: 0.8^(k-1) over positions k = 1, 2, ...)
+ *            at the first rejection instead of at the first position; the
+ *            ablation's hard cut-off gives zero weight after it.
  *
  * Readings where the pages are silent (each is listed in the design doc):
  *  - residual = normalise(max(0, p - q)) (the plain reading of "target minus what
@@ -48,6 +56,10 @@
  *    argmax of target row i; the emitted token is the argmax of row j;
  *  - draft_lens[b] outside [0, k_max] or a drafted id outside [0, V) for i < L
  *    -> the request is invalid: out_len = -1 and all its out_tokens = -1.
+ *
+ *  - acceptance simulation: E[j] = sum over m = 1..L of P(j >= m), with
+ *    P(j >= m) = prod_{l<m} a_l (independent uniforms); loss weight 1 for
+ *    i <= j and decay^(i - j) for i > j, 0 past the request's length.
  *
  * Near-tie flags (results are unique except inside these bands):
  *  ORACLE_FLAG_ACCEPT_TIE  |u_i - a_i| < 1e-5 at an examined position i <= j;
@@ -330,5 +342,74 @@ int oracle_spec_verify(int64_t B, int32_t k_max, int64_t V, int32_t dtype,
                            any_diag ? &diag : NULL, scratch, scratch + V,
                            scratch + 2 * V);
     free(scratch);
+    return 0;
+}
+
+/*
+ * Acceptance simulation over a batch [VAT-SIM], [VAT-W], from the per-position
+ * probabilities p[b*k_max + i] = p_i(x_i) and q[b*k_max + i] = q_i(x_i) that
+ * oracle_spec_verify returns (q = 1 for one-hot drafts):
+ *   out_a[b*k_max + i]  a_i = min(1, p_i / q_i) for i < L_b, NaN after;
+ *   out_e[b]            E[j] = sum_{m=1..L_b} prod_{l<m} a_l;
+ *   out_j[b]            (uniforms != NULL) the first i < L_b with
+ *                       u_i >= a_i (accept iff u < a), else L_b;
+ *   out_w[b*k_max + i]  (uniforms != NULL) 1 for i <= j, decay^(i-j) for
+ *                       j < i < L_b, 0 for i >= L_b.
+ * A request with L_b outside [0, k_max] or a drafted id outside [0, V) is
+ * invalid: out_j = -1, NaN elsewhere.  out_j / out_w may be NULL.
+ */
+int oracle_accept_sim(int64_t B, int32_t k_max, int64_t V, const int32_t *tokens,
+                      const int32_t *lens, const double *p, const double *q,
+                      const double *uniforms, double decay, double *out_a,
+                      double *out_e, int32_t *out_j, double *out_w)
+{
+    for (int64_t b = 0; b < B; ++b) {
+        const int32_t L = lens ? lens[b] : k_max;
+        int valid = L >= 0 && L <= k_max;
+        for (int32_t i = 0; valid && i < L; ++i)
+            if (tokens[b * k_max + i] < 0 || tokens[b * k_max + i] >= V)
+                valid = 0;
+        double *a = out_a + b * k_max;
+        if (!valid) {
+            for (int32_t i = 0; i < k_max; ++i) {
+                a[i] = NAN;
+                if (out_w)
+                    out_w[b * k_max + i] = NAN;
+            }
+            out_e[b] = NAN;
+            if (out_j)
+                out_j[b] = -1;
+            continue;
+        }
+        for (int32_t i = 0; i < k_max; ++i) {
+            if (i < L) {
+                const double r = p[b * k_max + i] / q[b * k_max + i];
+                a[i] = r > 1.0 ? 1.0 : r;
+            } else {
+                a[i] = NAN;
+            }
+        }
+        /* expected number of accepted drafts */
+        double e = 0.0, reach = 1.0; /* reach = P(j >= m) */
+        for (int32_t m = 1; m <= L; ++m) {
+            reach *= a[m - 1];
+            e += reach;
+        }
+        out_e[b] = e;
+        if (!uniforms)
+            continue;
+        int32_t j = L;
+        for (int32_t i = 0; i < L; ++i) {
+            if (!(uniforms[b * (k_max + 1) + i] < a[i])) {
+                j = i;
+                break;
+            }
+        }
+        if (out_j)
+            out_j[b] = j;
+        if (out_w)
+            for (int32_t i = 0; i < k_max; ++i)
+                out_w[b * k_max + i] = i >= L ? 0.0 : (i <= j ? 1.0 : pow(decay, (double)(i - j)));
+    }
     return 0;
 }

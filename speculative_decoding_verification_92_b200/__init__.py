@@ -22,7 +22,7 @@ from pathlib import Path
 
 __all__ = [
     "Status", "StatsKernel", "SpecVerifyError", "library", "workspace_bytes",
-    "spec_verify", "spec_verify_stats", "spec_verify_host", "host_staging_bytes",
+    "spec_verify", "spec_verify_stats", "spec_verify_accept_sim", "spec_verify_host", "host_staging_bytes",
     "abi_version", "F32", "BF16",
 ]
 
@@ -73,6 +73,8 @@ _SIGNATURES = {
                               _VP, ctypes.POINTER(_Options)]),
     "spec_verify_stats": (_I32, [ctypes.POINTER(_Shape), _VP, _VP, _VP, _VP, _F32, _VP, _VP, _VP, _VP, _VP, _SZ,
                                  _VP, ctypes.POINTER(_Options)]),
+    "spec_verify_accept_sim": (_I32, [ctypes.POINTER(_Shape), _VP, _VP, _VP, _VP, _VP, _F32, _F32, _VP, _VP, _VP, _VP,
+                                      _VP, _SZ, _VP]),
     "spec_verify_host_staging_bytes": (_SZ, [ctypes.POINTER(_Shape), _I32, _I32]),
     "spec_verify_host": (_I32, [ctypes.POINTER(_Shape), _VP, _VP, _VP, _VP, _VP, _F32, _I32, _VP, _VP, _VP, _SZ,
                                 _VP, _SZ, _VP]),
@@ -250,6 +252,37 @@ def spec_verify_stats(target, draft, tokens, lens, temperature=1.0, *, V=None, w
         _stream_handle(stream), ctypes.byref(opts))
     _check(st, "spec_verify_stats")
     return lse_t, lse_d, p, q
+
+
+def spec_verify_accept_sim(target, draft, tokens, lens, uniforms=None, temperature=1.0, decay=0.8, *, V=None,
+                           workspace=None, stream=None):
+    """Acceptance simulation (no draw): returns float32 / int32 device tensors
+    ``(accept_prob [B, k], expected_len [B], first_reject [B], weights [B, k])``
+    -- a_i = min(1, p_i/q_i) (NaN past the request's length), E[j], and, when
+    ``uniforms`` is given, the first rejection j and the per-position weights
+    (1 up to j, decay**(i - j) after, 0 past the length); the last two are
+    None without uniforms."""
+    torch = _torch()
+    B, k_max, V, dt, row_stride = _logit_shape(target, draft, V)
+    dev = target.device
+    a = torch.empty(B, k_max, dtype=torch.float32, device=dev)
+    e = torch.empty(B, dtype=torch.float32, device=dev)
+    j = torch.empty(B, dtype=torch.int32, device=dev) if uniforms is not None else None
+    w = torch.empty(B, k_max, dtype=torch.float32, device=dev) if uniforms is not None else None
+    shape = _shape(B, k_max, V, dt, row_stride)
+    lib = library()
+    if workspace is None:
+        workspace = torch.empty(max(lib.spec_verify_workspace_bytes(ctypes.byref(shape)), 256),
+                                dtype=torch.uint8, device=dev)
+    st = lib.spec_verify_accept_sim(
+        ctypes.byref(shape), _dev_ptr(target, what="target"), _dev_ptr(draft, what="draft"),
+        _dev_ptr(tokens, torch.int32, "draft_tokens"), _dev_ptr(lens, torch.int32, "draft_lens"),
+        _dev_ptr(uniforms, torch.float32, "uniforms"), float(temperature), float(decay),
+        a.data_ptr(), e.data_ptr(), None if j is None else j.data_ptr(), None if w is None else w.data_ptr(),
+        _dev_ptr(workspace, what="workspace"), workspace.numel() * workspace.element_size(),
+        _stream_handle(stream))
+    _check(st, "spec_verify_accept_sim")
+    return a, e, j, w
 
 
 def _host_ptr(t, dtype=None, what="tensor"):

@@ -223,6 +223,13 @@ struct Call {
     cudaStream_t stream;
     const sv_options* opts;
     bool stats_only;
+    // acceptance simulation (stats_only with the acceptance outputs)
+    bool accept_sim = false;
+    float decay = 0.f;
+    float* out_accept_prob = nullptr;
+    float* out_expected_len = nullptr;
+    int32_t* out_first_reject = nullptr;
+    float* out_weights = nullptr;
 };
 
 template <typename T>
@@ -276,6 +283,11 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     dp.scale = sp.scale;
     dp.greedy = greedy ? 1 : 0;
     dp.stats_only = a.stats_only ? 1 : 0;
+    dp.out_accept_prob = a.out_accept_prob;
+    dp.out_expected_len = a.out_expected_len;
+    dp.out_first_reject = a.out_first_reject;
+    dp.out_weights = a.out_weights;
+    dp.decay = a.decay;
     dp.rows_aligned = rows_aligned ? 1 : 0;
     dp.fast_draw = (rows_aligned && !greedy && !a.stats_only && int64_t(plan.CE) * plan.es <= kMaxChunkBytesFast) ? 1 : 0;
     {
@@ -305,7 +317,11 @@ sv_status run(const Call& a) {
     const bool greedy = a.greedy && !a.stats_only;
     if (!a.target) return SV_EINVAL;
     if (s.k_max > 0 && !a.tokens) return SV_EINVAL;
-    if (a.stats_only) {
+    if (a.accept_sim) {
+        if (!a.out_accept_prob || !a.out_expected_len) return SV_EINVAL;
+        if ((a.out_first_reject || a.out_weights) && !a.uniforms) return SV_EINVAL;
+        if (!(a.decay >= 0.f && a.decay <= 1.f)) return SV_EINVAL;
+    } else if (a.stats_only) {
         if (!a.out_lse_t) return SV_EINVAL;
     } else {
         if (!a.out_len || !a.out_tokens) return SV_EINVAL;
@@ -394,6 +410,24 @@ sv_status spec_verify_stats(const sv_shape* shape, const void* target_logits, co
                nullptr,        temperature,   false,        nullptr,      nullptr,
                out_lse_target, out_lse_draft, out_p,        out_q,        workspace,
                workspace_bytes, static_cast<cudaStream_t>(stream), opts, true};
+    return sv::run(a);
+}
+
+sv_status spec_verify_accept_sim(const sv_shape* shape, const void* target_logits, const void* draft_logits,
+                                 const int32_t* draft_tokens, const int32_t* draft_lens, const float* uniforms,
+                                 float temperature, float decay, float* out_accept_prob, float* out_expected_len,
+                                 int32_t* out_first_reject, float* out_weights, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    sv::Call a{shape,    target_logits, draft_logits, draft_tokens, draft_lens,
+               uniforms, temperature,   false,        nullptr,      nullptr,
+               nullptr,  nullptr,       nullptr,      nullptr,      workspace,
+               workspace_bytes, static_cast<cudaStream_t>(stream), nullptr, true};
+    a.accept_sim = true;
+    a.decay = decay;
+    a.out_accept_prob = out_accept_prob;
+    a.out_expected_len = out_expected_len;
+    a.out_first_reject = out_first_reject;
+    a.out_weights = out_weights;
     return sv::run(a);
 }
 

@@ -72,6 +72,11 @@ struct DrawParams {
     float* out_lse_d;
     float* out_p;
     float* out_q;
+    float* out_accept_prob;      // acceptance simulation outputs (stats mode), may be null
+    float* out_expected_len;
+    int32_t* out_first_reject;
+    float* out_weights;
+    float decay;
     int32_t b0;
     int32_t k_max;
     int32_t V;
@@ -148,6 +153,12 @@ __device__ __forceinline__ float block_scan_incl(float v, float* s_warp, float* 
 }
 
 enum DrawMode { kBonus = 0, kOneHot = 1, kResidual = 2 };
+
+// Acceptance probability min(1, p/q); NaN stays NaN (and then rejects).
+__device__ __forceinline__ float accept_prob(float p, float q) {
+    const float a = p / q;
+    return a > 1.f ? 1.f : a;
+}
 
 // Everything a segment pass needs to turn logits of row j into draw weights.
 struct WeightRow {
@@ -513,11 +524,18 @@ verify_draw_kernel(const DrawParams p) {
         if (c != 0) return;
         const float nan = __int_as_float(0x7fc00000);
         if (p.stats_only) {
-            for (int i = tid; i <= K; i += kDrawThreads) p.out_lse_t[int64_t(b) * (K + 1) + i] = nan;
+            for (int i = tid; i <= K; i += kDrawThreads)
+                if (p.out_lse_t) p.out_lse_t[int64_t(b) * (K + 1) + i] = nan;
             for (int i = tid; i < K; i += kDrawThreads) {
                 if (p.out_lse_d) p.out_lse_d[int64_t(b) * K + i] = nan;
                 if (p.out_p) p.out_p[int64_t(b) * K + i] = nan;
                 if (p.out_q) p.out_q[int64_t(b) * K + i] = nan;
+                if (p.out_accept_prob) p.out_accept_prob[int64_t(b) * K + i] = nan;
+                if (p.out_weights) p.out_weights[int64_t(b) * K + i] = nan;
+            }
+            if (tid == 0) {
+                if (p.out_expected_len) p.out_expected_len[b] = nan;
+                if (p.out_first_reject) p.out_first_reject[b] = code;
             }
         } else {
             for (int i = tid; i <= K; i += kDrawThreads) out_tok[i] = -1;
@@ -548,7 +566,7 @@ verify_draw_kernel(const DrawParams p) {
             if (i < L) {
                 s_p[i] = Logit<T>::load(trow_of(i), xr[k]);
                 if (has_draft) s_q[i] = Logit<T>::load(drow_of(i), xr[k]);
-                if (!p.stats_only) ur[k] = __ldg(u + i);
+                if (u) ur[k] = __ldg(u + i);
             }
         }
     }
@@ -615,9 +633,8 @@ verify_draw_kernel(const DrawParams p) {
             const float qi = has_draft ? exp2f(s_q[i] * p.scale - s_lse_d[i]) : 1.f;
             s_p[i] = pi;
             s_q[i] = qi;
-            float a = pi / qi;
-            a = a > 1.f ? 1.f : a;  // min(1, p/q); NaN stays NaN (rejects)
-            rej = p.stats_only ? false : !(ur[k] < a);
+            const float a = accept_prob(pi, qi);
+            rej = u ? !(ur[k] < a) : false;  // no uniforms (statistics only): no scan
         }
         if (rej) atomicMin(&s_first, i);
     }
@@ -626,12 +643,28 @@ verify_draw_kernel(const DrawParams p) {
     if (p.stats_only) {
         if (c == 0) {
             const float nan = __int_as_float(0x7fc00000);
+            const int j = s_first;  // L when no uniforms were given
             for (int i = tid; i <= K; i += kDrawThreads)
-                p.out_lse_t[int64_t(b) * (K + 1) + i] = i <= L ? s_lse_t[i] * kLn2 : nan;
+                if (p.out_lse_t) p.out_lse_t[int64_t(b) * (K + 1) + i] = i <= L ? s_lse_t[i] * kLn2 : nan;
             for (int i = tid; i < K; i += kDrawThreads) {
                 if (p.out_lse_d) p.out_lse_d[int64_t(b) * K + i] = (has_draft && i < L) ? s_lse_d[i] * kLn2 : nan;
                 if (p.out_p) p.out_p[int64_t(b) * K + i] = i < L ? s_p[i] : nan;
                 if (p.out_q) p.out_q[int64_t(b) * K + i] = i < L ? s_q[i] : nan;
+                if (p.out_accept_prob) p.out_accept_prob[int64_t(b) * K + i] = i < L ? accept_prob(s_p[i], s_q[i]) : nan;
+                if (p.out_weights)  // full weight up to the first rejection, the decay curve from there
+                    p.out_weights[int64_t(b) * K + i] = i >= L ? 0.f : (i <= j ? 1.f : powf(p.decay, float(i - j)));
+            }
+            if (tid == 0) {
+                if (p.out_first_reject) p.out_first_reject[b] = j;
+                if (p.out_expected_len) {
+                    // E[j] = sum_{m=1..L} P(j >= m), P(j >= m) = prod_{l<m} a_l
+                    float prod = 1.f, e = 0.f;
+                    for (int i = 0; i < L; ++i) {
+                        prod *= accept_prob(s_p[i], s_q[i]);
+                        e += prod;
+                    }
+                    p.out_expected_len[b] = e;
+                }
             }
         }
         return;

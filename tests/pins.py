@@ -443,6 +443,106 @@ def pin_invalid_requests(orc):
     assert j >= 0 and not flags & 4
 
 
+# ---------------------------------------------------------------------------
+# acceptance simulation ("今热点：让AI草稿模型学会"照镜子"", sections
+# "VAT怎么把"验收规则"塞进训练里" and "第二件事，改权重分配的锚点")
+
+def _sim(orc, p, q, lens=None, u=None, decay=0.8, tokens=None, V=100):
+    p = np.asarray(p, np.float64).reshape(1, -1)
+    q = np.asarray(q, np.float64).reshape(1, -1)
+    k = p.shape[1]
+    tokens = np.zeros((1, k), np.int32) if tokens is None else np.asarray(tokens, np.int32).reshape(1, k)
+    lens = None if lens is None else np.asarray([lens], np.int32)
+    u = None if u is None else np.asarray(u, np.float64).reshape(1, k + 1)
+    r = orc.accept_sim(p, q, tokens, lens, u, decay, V=V)
+    return {key: (None if v is None else v[0]) for key, v in r.items()}
+
+
+def pin_accept_sim_closed_forms(orc):
+    # the page's worked ratios: q=0.9, pi=0.95 -> 1; q=0.9, pi=0.1 -> 1/9
+    r = _sim(orc, [0.95, 0.1], [0.9, 0.9])
+    assert r["a"][0] == 1.0 and abs(r["a"][1] - 1.0 / 9.0) < 1e-15
+    # constant a = c: E[j] = c (1 - c^L) / (1 - c)
+    for c, L in ((0.5, 3), (0.9, 12), (0.25, 1), (0.7, 24)):
+        r = _sim(orc, [c] * L, [1.0] * L)
+        want = c * (1 - c ** L) / (1 - c)
+        assert abs(r["e"] - want) < 1e-12 * max(1.0, want), (c, L, r["e"], want)
+    # certain acceptance: E = L; a zero at position 0: E = 0
+    assert _sim(orc, [0.3, 0.2, 0.9], [0.1, 0.2, 0.5])["e"] == 3.0
+    assert _sim(orc, [0.0, 1.0, 1.0], [0.5, 0.5, 0.5])["e"] == 0.0
+    # positions past the length carry NaN, the expectation stops at L
+    r = _sim(orc, [0.5, 0.5, 0.5, 0.5], [1.0] * 4, lens=2)
+    assert np.isnan(r["a"][2:]).all() and abs(r["e"] - 0.75) < 1e-15
+
+
+def pin_accept_sim_expectation_by_enumeration(orc):
+    """E[j] against the distribution of the first rejection, built by
+    enumerating every accept / reject pattern of independent Bernoulli(a_l)."""
+    rng = np.random.default_rng(7)
+    for L in (1, 2, 5, 9):
+        a = rng.uniform(0.05, 1.0, L)
+        a[rng.integers(0, L)] = 1.0
+        want = 0.0
+        for mask in range(1 << L):
+            prob, first = 1.0, L
+            for l in range(L):
+                ok = (mask >> l) & 1
+                prob *= a[l] if ok else 1.0 - a[l]
+                if not ok and first == L:
+                    first = l
+            want += prob * first
+        r = _sim(orc, a, np.ones(L))
+        assert abs(r["e"] - want) < 1e-12, (L, r["e"], want)
+
+
+def pin_accept_sim_first_rejection_and_weights(orc):
+    # the page's example: ten drafts pass, the eleventh is rejected -> the
+    # first ten keep full weight, the decay curve starts at the rejection
+    L = 16
+    p, q = np.full(L, 0.5), np.ones(L)
+    u = np.zeros(L + 1)
+    u[10] = 0.75                     # 0.75 >= a = 0.5: first rejection at i = 10
+    u[11:] = 0.99                    # later uniforms do not matter
+    r = _sim(orc, p, q, u=u, decay=0.8)
+    assert r["j"] == 10
+    assert np.array_equal(r["w"][:11], np.ones(11))
+    assert np.allclose(r["w"][11:], 0.8 ** np.arange(1, L - 10), rtol=1e-15, atol=0)
+    # the ablation's hard cut-off and a flat curve
+    assert np.array_equal(_sim(orc, p, q, u=u, decay=0.0)["w"], np.r_[np.ones(11), np.zeros(L - 11)])
+    assert np.array_equal(_sim(orc, p, q, u=u, decay=1.0)["w"], np.ones(L))
+    # all accepted: j = L, full weight; padding weight 0
+    r = _sim(orc, p, q, lens=5, u=np.zeros(L + 1))
+    assert r["j"] == 5 and np.array_equal(r["w"], np.r_[np.ones(5), np.zeros(L - 5)])
+    # u == a rejects (accept iff u < a)
+    assert _sim(orc, [0.5, 1.0], [1.0, 1.0], u=[0.5, 0.0, 0.0])["j"] == 0
+    # invalid requests: -1 and NaN
+    r = _sim(orc, [0.5, 0.5], [1.0, 1.0], u=[0, 0, 0], tokens=[1, 100], V=100)
+    assert r["j"] == -1 and np.isnan(r["e"]) and np.isnan(r["a"]).all()
+
+
+def pin_accept_sim_matches_verify_and_monte_carlo(orc):
+    """j equals the verification rule's j on the same inputs, and the mean of
+    j over independent uniform draws converges to E[j]."""
+    rng = np.random.default_rng(11)
+    V, k = 12, 6
+    z = rng.normal(0, 1.5, (k + 1, V)).astype(np.float32)
+    y = (z[:k] + rng.normal(0, 0.8, (k, V))).astype(np.float32)
+    toks = [int(np.argmax(y[i] + rng.gumbel(size=V))) for i in range(k)]
+    _, _, _, out = run1(orc, z, y, toks, np.zeros(k + 1), diag=True)
+    p, q = out["p"][0], out["q"][0]
+    js = []
+    for _ in range(4000):
+        u = rng.random(k + 1)
+        j_ver, _, flags = run1(orc, z, y, toks, u)
+        r = _sim(orc, p, q, u=u, tokens=toks, V=V)
+        if not flags & 1:
+            assert r["j"] == j_ver
+        js.append(r["j"])
+    e = _sim(orc, p, q, tokens=toks, V=V)["e"]
+    sd = np.std(js) / math.sqrt(len(js))
+    assert abs(np.mean(js) - e) < 5 * sd + 1e-9, (np.mean(js), e, sd)
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_lse_closed_forms,
@@ -460,6 +560,10 @@ ALL_PINS = [
     pin_sequential_rule,
     pin_greedy,
     pin_invalid_requests,
+    pin_accept_sim_closed_forms,
+    pin_accept_sim_expectation_by_enumeration,
+    pin_accept_sim_first_rejection_and_weights,
+    pin_accept_sim_matches_verify_and_monte_carlo,
 ]
 
 

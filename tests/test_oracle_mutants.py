@@ -50,6 +50,14 @@ MUTANTS = [
      "    /* else j == L: bonus draw from p_L [NG-PIPE]; w already holds p_L. */",
      "    else { (void)row_log_sum_exp(TROW(0), dtype, V, T, ell_t);\n"
      "      for (int64_t v = 0; v < V; ++v) w[v] = exp(ell_t[v] - lse_t_row[0]); }"),
+    ("expected length counts the reach before the position",
+     "            reach *= a[m - 1];\n            e += reach;", "            e += reach;\n            reach *= a[m - 1];"),
+    ("simulated acceptance accepts on u == a",
+     "if (!(uniforms[b * (k_max + 1) + i] < a[i])) {", "if (!(uniforms[b * (k_max + 1) + i] <= a[i])) {"),
+    ("decay starts at the first position",
+     "(i <= j ? 1.0 : pow(decay, (double)(i - j)))", "pow(decay, (double)i)"),
+    ("acceptance probability not clamped at one",
+     "                a[i] = r > 1.0 ? 1.0 : r;", "                a[i] = r;"),
 ]
 
 
