@@ -2,7 +2,8 @@
 
 ``python -m speculative_decoding_verification_92_b200.build`` (or
 ``build()``) compiles ``csrc/spec_verify.cu`` (which includes the kernel
-headers) into ``speculative_decoding_verification_92_b200/libspecverify.so``.
+headers) and the host-side ``csrc/*.cpp`` into
+``speculative_decoding_verification_92_b200/libspecverify.so``.
 The library is rebuilt only when the sources or the public header change
 (content hash stored beside the library).
 """
@@ -31,7 +32,25 @@ def _nvcc() -> str:
 
 
 def sources() -> list[Path]:
-    return sorted(CSRC.glob("*.cu")) + sorted(CSRC.glob("*.cuh")) + sorted(INCLUDE.glob("*.h"))
+    return (sorted(CSRC.glob("*.cu")) + sorted(CSRC.glob("*.cuh")) + sorted(CSRC.glob("*.cpp"))
+            + sorted(INCLUDE.glob("*.h")))
+
+
+def kernel_sources() -> list[Path]:
+    """The sources the GPU kernels and their launches are built from (the
+    host-only components in csrc/*.cpp and include/sv_host.h excluded)."""
+    return sorted(CSRC.glob("*.cu")) + sorted(CSRC.glob("*.cuh")) + [INCLUDE / "spec_verify.h"]
+
+
+def kernel_source_hash() -> str:
+    """Hash of kernel_sources(): profiles of a kernel stay valid while it is
+    unchanged."""
+    h = hashlib.sha256()
+    for s in kernel_sources():
+        h.update(s.name.encode())
+        h.update(s.read_bytes())
+    h.update(" ".join(ARCH).encode())
+    return h.hexdigest()
 
 
 def source_hash() -> str:
@@ -60,7 +79,7 @@ def nvcc_command(out: Path, extra=()) -> list[str]:
     return [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--shared",
             "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
             "-I", str(INCLUDE), "-I", str(CSRC), *extra,
-            "-o", str(out), str(CSRC / "spec_verify.cu")]
+            "-o", str(out), str(CSRC / "spec_verify.cu"), *[str(p) for p in sorted(CSRC.glob("*.cpp"))]]
 
 
 def build(force: bool = False, verbose: bool = False, extra=(), out: Path | None = None) -> Path:

@@ -1,0 +1,544 @@
+// sv_host.cpp -- host-side components declared in include/sv_host.h: the
+// per-prompt n-gram drafter, the suffix drafter with frequency scoring, the
+// fan-out prefetch budget, the draft-length controller, the speculation
+// switch and the length-aware budgets.  Plain C++17 on host memory; nothing
+// here touches a GPU.  The rules each function follows are stated in the
+// header, with the page and section they come from.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <deque>
+#include <limits>
+#include <new>
+#include <numeric>
+#include <unordered_map>
+#include <vector>
+
+#include "spec_verify.h"
+#include "sv_host.h"
+
+namespace {
+
+// 64-bit FNV-1a over a run of token ids (n-gram / context keys; every hit is
+// confirmed by comparing the tokens, so collisions cost time, never results).
+uint64_t hash_tokens(const int32_t* t, int64_t n) {
+    uint64_t h = 1469598103934665603ull ^ static_cast<uint64_t>(n);
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t v = static_cast<uint32_t>(t[i]);
+        for (int b = 0; b < 4; ++b) {
+            h ^= (v >> (8 * b)) & 0xffu;
+            h *= 1099511628211ull;
+        }
+    }
+    return h;
+}
+
+}  // namespace
+
+// ===========================================================================
+// Per-prompt n-gram drafter.
+
+struct sv_ngram {
+    struct Rollout {
+        int64_t step;
+        std::vector<int32_t> tok;
+        // key of the n-gram tok[p-n .. p) (n = 1..max_n) -> every p, ascending;
+        // p is the position right after the n-gram (where a continuation starts)
+        std::unordered_map<uint64_t, std::vector<int32_t>> ends;
+    };
+    int32_t max_n = 6;
+    int32_t window = 4;
+    int64_t step = 0;
+    bool started = false;
+    // per prompt, oldest first (so newest = back)
+    std::unordered_map<int64_t, std::deque<Rollout>> prompts;
+};
+
+namespace {
+
+struct Occurrence {
+    const sv_ngram::Rollout* r = nullptr;
+    int64_t p = -1;  // continuation start
+};
+
+// The last n context tokens followed by at least one token in rollout r:
+// the latest such position, or -1.
+int64_t latest_in(const sv_ngram::Rollout& r, const int32_t* key, int32_t n, uint64_t h) {
+    auto it = r.ends.find(h);
+    if (it == r.ends.end()) return -1;
+    const std::vector<int32_t>& ps = it->second;
+    for (auto q = ps.rbegin(); q != ps.rend(); ++q) {
+        const int64_t p = *q;
+        if (p >= static_cast<int64_t>(r.tok.size())) continue;  // nothing follows
+        if (std::memcmp(r.tok.data() + p - n, key, sizeof(int32_t) * n) == 0) return p;
+    }
+    return -1;
+}
+
+// Longest n with an occurrence; fills the most recent occurrence.
+int32_t longest_match(const sv_ngram& t, const std::deque<sv_ngram::Rollout>& rs, const int32_t* ctx,
+                      int64_t n_ctx, Occurrence* occ) {
+    const int32_t top = static_cast<int32_t>(std::min<int64_t>(t.max_n, n_ctx));
+    for (int32_t n = top; n >= 1; --n) {
+        const int32_t* key = ctx + n_ctx - n;
+        const uint64_t h = hash_tokens(key, n);
+        for (auto r = rs.rbegin(); r != rs.rend(); ++r) {
+            const int64_t p = latest_in(*r, key, n, h);
+            if (p >= 0) {
+                occ->r = &*r;
+                occ->p = p;
+                return n;
+            }
+        }
+    }
+    return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+sv_ngram* sv_ngram_create(int32_t max_n, int32_t window) {
+    if (max_n < 1 || max_n > 16 || window < 1) return nullptr;
+    sv_ngram* t = new (std::nothrow) sv_ngram;
+    if (!t) return nullptr;
+    t->max_n = max_n;
+    t->window = window;
+    return t;
+}
+
+void sv_ngram_destroy(sv_ngram* t) { delete t; }
+
+void sv_ngram_begin_step(sv_ngram* t) {
+    if (!t) return;
+    if (t->started) ++t->step;
+    t->started = true;
+    for (auto it = t->prompts.begin(); it != t->prompts.end();) {
+        auto& rs = it->second;
+        while (!rs.empty() && rs.front().step <= t->step - t->window) rs.pop_front();
+        if (rs.empty()) it = t->prompts.erase(it);
+        else ++it;
+    }
+}
+
+int32_t sv_ngram_add(sv_ngram* t, int64_t prompt_id, const int32_t* tokens, int64_t n) {
+    if (!t || n < 0 || (n > 0 && !tokens) || n > std::numeric_limits<int32_t>::max()) return -1;
+    if (!t->started) sv_ngram_begin_step(t);
+    sv_ngram::Rollout r;
+    r.step = t->step;
+    r.tok.assign(tokens, tokens + n);
+    for (int64_t p = 1; p <= n; ++p)
+        for (int32_t k = 1; k <= t->max_n && k <= p; ++k)
+            r.ends[hash_tokens(tokens + p - k, k)].push_back(static_cast<int32_t>(p));
+    t->prompts[prompt_id].push_back(std::move(r));
+    return 0;
+}
+
+int32_t sv_ngram_draft(const sv_ngram* t, int64_t prompt_id, const int32_t* context, int64_t n, int32_t k,
+                       int32_t* out) {
+    if (!t || n < 0 || (n > 0 && !context) || k < 0 || (k > 0 && !out)) return -1;
+    auto it = t->prompts.find(prompt_id);
+    if (it == t->prompts.end() || n == 0 || k == 0) return 0;
+    Occurrence occ;
+    if (longest_match(*t, it->second, context, n, &occ) == 0) return 0;
+    const int64_t avail = static_cast<int64_t>(occ.r->tok.size()) - occ.p;
+    const int32_t m = static_cast<int32_t>(std::min<int64_t>(k, avail));
+    std::memcpy(out, occ.r->tok.data() + occ.p, sizeof(int32_t) * m);
+    return m;
+}
+
+int32_t sv_ngram_candidates(const sv_ngram* t, int64_t prompt_id, const int32_t* context, int64_t n, int32_t f,
+                            int32_t* out) {
+    if (!t || n < 0 || (n > 0 && !context) || f < 0 || (f > 0 && !out)) return -1;
+    auto it = t->prompts.find(prompt_id);
+    if (it == t->prompts.end() || n == 0 || f == 0) return 0;
+    Occurrence occ;
+    const int32_t nm = longest_match(*t, it->second, context, n, &occ);
+    if (nm == 0) return 0;
+    // every occurrence of the matched n-gram, newest first: count followers
+    // and remember the order of their most recent occurrence
+    const int32_t* key = context + n - nm;
+    const uint64_t h = hash_tokens(key, nm);
+    struct Cand { int32_t tok; int64_t count; int64_t first_seen; };
+    std::vector<Cand> cands;
+    std::unordered_map<int32_t, size_t> slot;
+    int64_t order = 0;
+    const auto& rs = it->second;
+    for (auto r = rs.rbegin(); r != rs.rend(); ++r) {
+        auto e = r->ends.find(h);
+        if (e == r->ends.end()) continue;
+        for (auto q = e->second.rbegin(); q != e->second.rend(); ++q) {
+            const int64_t p = *q;
+            if (p >= static_cast<int64_t>(r->tok.size())) continue;
+            if (std::memcmp(r->tok.data() + p - nm, key, sizeof(int32_t) * nm) != 0) continue;
+            const int32_t nxt = r->tok[p];
+            auto s = slot.find(nxt);
+            if (s == slot.end()) {
+                slot.emplace(nxt, cands.size());
+                cands.push_back({nxt, 1, order});
+            } else {
+                ++cands[s->second].count;
+            }
+            ++order;
+        }
+    }
+    std::stable_sort(cands.begin(), cands.end(), [](const Cand& a, const Cand& b) {
+        return a.count != b.count ? a.count > b.count : a.first_seen < b.first_seen;
+    });
+    const int32_t m = static_cast<int32_t>(std::min<size_t>(f, cands.size()));
+    for (int32_t i = 0; i < m; ++i) out[i] = cands[i].tok;
+    return m;
+}
+
+int64_t sv_ngram_rollouts(const sv_ngram* t) {
+    if (!t) return -1;
+    int64_t n = 0;
+    for (const auto& kv : t->prompts) n += static_cast<int64_t>(kv.second.size());
+    return n;
+}
+
+int64_t sv_ngram_tokens(const sv_ngram* t) {
+    if (!t) return -1;
+    int64_t n = 0;
+    for (const auto& kv : t->prompts)
+        for (const auto& r : kv.second) n += static_cast<int64_t>(r.tok.size());
+    return n;
+}
+
+}  // extern "C"
+
+// ===========================================================================
+// Suffix drafter with frequency scoring.
+
+struct sv_suffix {
+    struct Context {
+        std::vector<int32_t> ctx;                    // the context tokens
+        std::unordered_map<int32_t, int64_t> next;   // follower -> count
+    };
+    struct Problem {
+        std::unordered_map<int64_t, std::vector<int32_t>> seqs;
+        std::unordered_map<uint64_t, std::vector<Context>> table;  // hash of ctx -> contexts
+    };
+    int32_t max_depth = 8;
+    std::unordered_map<int64_t, Problem> problems;
+};
+
+namespace {
+
+const sv_suffix::Context* find_context(const sv_suffix::Problem& pb, const int32_t* c, int32_t d) {
+    auto it = pb.table.find(hash_tokens(c, d));
+    if (it == pb.table.end()) return nullptr;
+    for (const auto& e : it->second)
+        if (static_cast<int32_t>(e.ctx.size()) == d && std::memcmp(e.ctx.data(), c, sizeof(int32_t) * d) == 0)
+            return &e;
+    return nullptr;
+}
+
+// Longest d <= max_depth with a count table for the last d tokens of c[0..n).
+const sv_suffix::Context* longest_context(const sv_suffix& t, const sv_suffix::Problem& pb, const int32_t* c,
+                                          int64_t n) {
+    const int32_t top = static_cast<int32_t>(std::min<int64_t>(t.max_depth, n));
+    for (int32_t d = top; d >= 1; --d) {
+        const sv_suffix::Context* e = find_context(pb, c + n - d, d);
+        if (e) return e;
+    }
+    return nullptr;
+}
+
+// Most frequent follower, ties to the lowest id.
+int32_t top_follower(const sv_suffix::Context& e) {
+    int32_t best = 0;
+    int64_t best_n = -1;
+    for (const auto& kv : e.next)
+        if (kv.second > best_n || (kv.second == best_n && kv.first < best)) {
+            best = kv.first;
+            best_n = kv.second;
+        }
+    return best;
+}
+
+}  // namespace
+
+extern "C" {
+
+sv_suffix* sv_suffix_create(int32_t max_depth) {
+    if (max_depth < 1 || max_depth > 64) return nullptr;
+    sv_suffix* t = new (std::nothrow) sv_suffix;
+    if (!t) return nullptr;
+    t->max_depth = max_depth;
+    return t;
+}
+
+void sv_suffix_destroy(sv_suffix* t) { delete t; }
+
+void sv_suffix_clear(sv_suffix* t) {
+    if (t) t->problems.clear();
+}
+
+int32_t sv_suffix_append(sv_suffix* t, int64_t problem_id, int64_t seq_id, const int32_t* tokens, int64_t m) {
+    if (!t || m < 0 || (m > 0 && !tokens)) return -1;
+    sv_suffix::Problem& pb = t->problems[problem_id];
+    std::vector<int32_t>& seq = pb.seqs[seq_id];
+    for (int64_t i = 0; i < m; ++i) {
+        const int32_t tok = tokens[i];
+        const int64_t n = static_cast<int64_t>(seq.size());
+        for (int32_t d = 1; d <= t->max_depth && d <= n; ++d) {
+            const int32_t* c = seq.data() + n - d;
+            auto& bucket = pb.table[hash_tokens(c, d)];
+            sv_suffix::Context* e = nullptr;
+            for (auto& x : bucket)
+                if (static_cast<int32_t>(x.ctx.size()) == d && std::memcmp(x.ctx.data(), c, sizeof(int32_t) * d) == 0) {
+                    e = &x;
+                    break;
+                }
+            if (!e) {
+                bucket.push_back(sv_suffix::Context{std::vector<int32_t>(c, c + d), {}});
+                e = &bucket.back();
+            }
+            ++e->next[tok];
+        }
+        seq.push_back(tok);
+    }
+    return 0;
+}
+
+int32_t sv_suffix_draft(const sv_suffix* t, int64_t problem_id, const int32_t* context, int64_t n, int32_t k,
+                        int32_t* out) {
+    if (!t || n < 0 || (n > 0 && !context) || k < 0 || (k > 0 && !out)) return -1;
+    auto it = t->problems.find(problem_id);
+    if (it == t->problems.end() || k == 0) return 0;
+    // the draft extends the context: keep the last max_depth tokens of both
+    std::vector<int32_t> ctx(context + std::max<int64_t>(0, n - t->max_depth), context + n);
+    int32_t m = 0;
+    while (m < k) {
+        const sv_suffix::Context* e = longest_context(*t, it->second, ctx.data(), static_cast<int64_t>(ctx.size()));
+        if (!e) break;
+        const int32_t tok = top_follower(*e);
+        out[m++] = tok;
+        ctx.push_back(tok);
+        if (static_cast<int32_t>(ctx.size()) > t->max_depth) ctx.erase(ctx.begin());
+    }
+    return m;
+}
+
+int32_t sv_suffix_candidates(const sv_suffix* t, int64_t problem_id, const int32_t* context, int64_t n, int32_t f,
+                             int32_t* out) {
+    if (!t || n < 0 || (n > 0 && !context) || f < 0 || (f > 0 && !out)) return -1;
+    auto it = t->problems.find(problem_id);
+    if (it == t->problems.end() || f == 0) return 0;
+    const sv_suffix::Context* e = longest_context(*t, it->second, context, n);
+    if (!e) return 0;
+    std::vector<std::pair<int32_t, int64_t>> c(e->next.begin(), e->next.end());
+    std::sort(c.begin(), c.end(), [](const auto& a, const auto& b) {
+        return a.second != b.second ? a.second > b.second : a.first < b.first;
+    });
+    const int32_t m = static_cast<int32_t>(std::min<size_t>(f, c.size()));
+    for (int32_t i = 0; i < m; ++i) out[i] = c[i].first;
+    return m;
+}
+
+}  // extern "C"
+
+// ===========================================================================
+// Fan-out prefetch budget.
+
+struct sv_prefetch {
+    int32_t k = 0, fmax = 1, window = 1;
+    std::deque<std::pair<int32_t, int32_t>> obs;  // (j, rank), oldest first
+};
+
+namespace {
+
+// P(j) and c_j(f) over the window; returns the observation count.
+int32_t estimates(const sv_prefetch& p, std::vector<double>* P, std::vector<double>* cov) {
+    const int32_t K1 = p.k + 1, F1 = p.fmax + 1;
+    P->assign(K1, 0.0);
+    cov->assign(size_t(K1) * F1, 0.0);
+    const int32_t n = static_cast<int32_t>(p.obs.size());
+    if (n == 0) return 0;
+    std::vector<int64_t> cnt(K1, 0), hits(size_t(K1) * F1, 0), pooled(F1, 0);
+    for (const auto& o : p.obs) {
+        ++cnt[o.first];
+        for (int32_t f = 1; f <= p.fmax; ++f)
+            if (o.second >= 0 && o.second < f) {
+                ++hits[size_t(o.first) * F1 + f];
+                ++pooled[f];
+            }
+    }
+    for (int32_t j = 0; j < K1; ++j) {
+        (*P)[j] = double(cnt[j]) / n;
+        for (int32_t f = 1; f <= p.fmax; ++f)
+            (*cov)[size_t(j) * F1 + f] = cnt[j] ? double(hits[size_t(j) * F1 + f]) / cnt[j] : double(pooled[f]) / n;
+    }
+    return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+sv_prefetch* sv_prefetch_create(int32_t k, int32_t fmax, int32_t window) {
+    if (k < 0 || fmax < 1 || window < 1) return nullptr;
+    sv_prefetch* p = new (std::nothrow) sv_prefetch;
+    if (!p) return nullptr;
+    p->k = k;
+    p->fmax = fmax;
+    p->window = window;
+    return p;
+}
+
+void sv_prefetch_destroy(sv_prefetch* p) { delete p; }
+
+int32_t sv_prefetch_observe(sv_prefetch* p, int32_t j, int32_t b_rank) {
+    if (!p || j < 0 || j > p->k || b_rank < -1) return -1;
+    p->obs.emplace_back(j, b_rank >= p->fmax ? -1 : b_rank);
+    while (static_cast<int32_t>(p->obs.size()) > p->window) p->obs.pop_front();
+    return 0;
+}
+
+int32_t sv_prefetch_estimates(const sv_prefetch* p, double* P_j, double* coverage) {
+    if (!p) return -1;
+    std::vector<double> P, cov;
+    const int32_t n = estimates(*p, &P, &cov);
+    if (P_j) std::copy(P.begin(), P.end(), P_j);
+    if (coverage) std::copy(cov.begin(), cov.end(), coverage);
+    return n;
+}
+
+double sv_prefetch_allocate(const sv_prefetch* p, int32_t budget, int32_t* out_f) {
+    if (!p || !out_f) return -1.0;
+    const int32_t K1 = p->k + 1, F1 = p->fmax + 1;
+    std::fill(out_f, out_f + K1, 0);
+    std::vector<double> P, cov;
+    if (estimates(*p, &P, &cov) == 0) return 0.0;
+    double total = 0.0;
+    for (int32_t spent = 0; spent < budget; ++spent) {
+        int32_t best = -1;
+        double best_gain = 0.0;
+        for (int32_t j = 0; j < K1; ++j) {
+            if (out_f[j] >= p->fmax) continue;
+            const double g = P[j] * (cov[size_t(j) * F1 + out_f[j] + 1] - cov[size_t(j) * F1 + out_f[j]]);
+            if (g > best_gain) {  // strict: ties keep the lower j
+                best_gain = g;
+                best = j;
+            }
+        }
+        if (best < 0) break;
+        ++out_f[best];
+        total += best_gain;
+    }
+    return total;
+}
+
+// ===========================================================================
+// Draft-length controller, block efficiency, speculation switch.
+
+}  // extern "C"
+
+struct sv_draft_len {
+    std::vector<int32_t> lengths;
+    double up = 0.7, down = 0.4;
+    int32_t patience = 2;
+    int32_t idx = 0, up_run = 0, down_run = 0;
+};
+
+extern "C" {
+
+sv_draft_len* sv_draft_len_create(const int32_t* lengths, int32_t n_lengths, double up_frac, double down_frac,
+                                  int32_t patience) {
+    if (!lengths || n_lengths < 1 || n_lengths > 64 || patience < 1) return nullptr;
+    if (!(down_frac >= 0.0 && down_frac <= up_frac && up_frac <= 1.0)) return nullptr;
+    for (int32_t i = 0; i < n_lengths; ++i)
+        if (lengths[i] < 1 || (i > 0 && lengths[i] <= lengths[i - 1])) return nullptr;
+    sv_draft_len* c = new (std::nothrow) sv_draft_len;
+    if (!c) return nullptr;
+    c->lengths.assign(lengths, lengths + n_lengths);
+    c->up = up_frac;
+    c->down = down_frac;
+    c->patience = patience;
+    return c;
+}
+
+void sv_draft_len_destroy(sv_draft_len* c) { delete c; }
+
+int32_t sv_draft_len_current(const sv_draft_len* c) { return c ? c->lengths[c->idx] : -1; }
+
+int32_t sv_draft_len_update(sv_draft_len* c, double tau) {
+    if (!c) return -1;
+    const double r = tau / double(c->lengths[c->idx] + 1);
+    // NaN (no valid request this step) extends neither streak
+    c->up_run = r >= c->up ? c->up_run + 1 : 0;
+    c->down_run = r < c->down ? c->down_run + 1 : 0;
+    if (c->up_run >= c->patience && c->idx + 1 < static_cast<int32_t>(c->lengths.size())) {
+        ++c->idx;
+        c->up_run = c->down_run = 0;
+    } else if (c->down_run >= c->patience && c->idx > 0) {
+        --c->idx;
+        c->up_run = c->down_run = 0;
+    }
+    return c->lengths[c->idx];
+}
+
+double sv_block_efficiency(const int32_t* accept_len, int64_t n) {
+    if (!accept_len || n <= 0) return std::numeric_limits<double>::quiet_NaN();
+    double s = 0.0;
+    int64_t m = 0;
+    for (int64_t i = 0; i < n; ++i)
+        if (accept_len[i] >= 0) {
+            s += double(accept_len[i]) + 1.0;
+            ++m;
+        }
+    return m ? s / double(m) : std::numeric_limits<double>::quiet_NaN();
+}
+
+int32_t sv_spec_switch(int32_t* state, double predicted_speedup, double threshold) {
+    if (!state) return -1;
+    if (*state == 0 && predicted_speedup > threshold) *state = 1;
+    return *state != 0 ? 1 : 0;
+}
+
+// ===========================================================================
+// Length-aware budgets.
+
+}  // extern "C"
+
+namespace {
+
+std::vector<int64_t> longest_first(const double* len, int64_t n) {
+    std::vector<int64_t> order(static_cast<size_t>(n));
+    std::iota(order.begin(), order.end(), int64_t(0));
+    std::stable_sort(order.begin(), order.end(), [len](int64_t a, int64_t b) { return len[a] > len[b]; });
+    return order;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t sv_length_classes(const double* predicted_len, int64_t n, const int32_t budgets[3], int32_t* out_class,
+                          int32_t* out_budget) {
+    if (n < 0 || (n > 0 && (!predicted_len || !budgets || !out_class || !out_budget))) return -1;
+    for (int64_t i = 0; i < n; ++i)
+        if (std::isnan(predicted_len[i])) return -1;
+    const std::vector<int64_t> order = longest_first(predicted_len, n);
+    const int64_t third = n / 3;
+    for (int64_t r = 0; r < n; ++r) {
+        const int64_t i = order[static_cast<size_t>(r)];
+        const int32_t cls = r < third ? 2 : (r >= n - third ? 0 : 1);
+        out_class[i] = cls;
+        out_budget[i] = budgets[cls];
+    }
+    return 0;
+}
+
+int32_t sv_interleave_ranks(const double* predicted_len, int64_t n, int32_t world_size, int32_t* out_rank) {
+    if (n < 0 || world_size < 1 || (n > 0 && (!predicted_len || !out_rank))) return -1;
+    for (int64_t i = 0; i < n; ++i)
+        if (std::isnan(predicted_len[i])) return -1;
+    const std::vector<int64_t> order = longest_first(predicted_len, n);
+    for (int64_t r = 0; r < n; ++r) out_rank[order[static_cast<size_t>(r)]] = static_cast<int32_t>(r % world_size);
+    return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,227 @@
+"""ctypes binding of the host-side components in ``include/sv_host.h``.
+
+Every class wraps one C handle of ``libspecverify.so`` (argument marshalling
+only; the logic lives in ``csrc/sv_host.cpp``).  Token sequences are passed
+as int32 numpy arrays (anything ``numpy.asarray`` accepts)."""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import library
+
+_I32, _I64, _F64, _VP = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+
+_HOST_SIGNATURES = {
+    "sv_ngram_create": (_VP, [_I32, _I32]),
+    "sv_ngram_destroy": (None, [_VP]),
+    "sv_ngram_begin_step": (None, [_VP]),
+    "sv_ngram_add": (_I32, [_VP, _I64, _VP, _I64]),
+    "sv_ngram_draft": (_I32, [_VP, _I64, _VP, _I64, _I32, _VP]),
+    "sv_ngram_candidates": (_I32, [_VP, _I64, _VP, _I64, _I32, _VP]),
+    "sv_ngram_rollouts": (_I64, [_VP]),
+    "sv_ngram_tokens": (_I64, [_VP]),
+    "sv_suffix_create": (_VP, [_I32]),
+    "sv_suffix_destroy": (None, [_VP]),
+    "sv_suffix_clear": (None, [_VP]),
+    "sv_suffix_append": (_I32, [_VP, _I64, _I64, _VP, _I64]),
+    "sv_suffix_draft": (_I32, [_VP, _I64, _VP, _I64, _I32, _VP]),
+    "sv_suffix_candidates": (_I32, [_VP, _I64, _VP, _I64, _I32, _VP]),
+    "sv_prefetch_create": (_VP, [_I32, _I32, _I32]),
+    "sv_prefetch_destroy": (None, [_VP]),
+    "sv_prefetch_observe": (_I32, [_VP, _I32, _I32]),
+    "sv_prefetch_estimates": (_I32, [_VP, _VP, _VP]),
+    "sv_prefetch_allocate": (_F64, [_VP, _I32, _VP]),
+    "sv_draft_len_create": (_VP, [_VP, _I32, _F64, _F64, _I32]),
+    "sv_draft_len_destroy": (None, [_VP]),
+    "sv_draft_len_current": (_I32, [_VP]),
+    "sv_draft_len_update": (_I32, [_VP, _F64]),
+    "sv_block_efficiency": (_F64, [_VP, _I64]),
+    "sv_spec_switch": (_I32, [_VP, _F64, _F64]),
+    "sv_length_classes": (_I32, [_VP, _I64, _VP, _VP, _VP]),
+    "sv_interleave_ranks": (_I32, [_VP, _I64, _I32, _VP]),
+}
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = library()
+        for name, (res, args) in _HOST_SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _tok(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32).reshape(-1))
+
+
+class _Handle:
+    _destroy = ""
+
+    def __init__(self, h):
+        if not h:
+            raise ValueError(f"{type(self).__name__}: invalid arguments")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            getattr(_L(), self._destroy)(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class NgramDrafter(_Handle):
+    """Per-prompt n-gram drafter over the rollouts of the last ``window``
+    training steps (longest match up to ``max_n``, most recent occurrence)."""
+    _destroy = "sv_ngram_destroy"
+
+    def __init__(self, max_n: int = 6, window: int = 4):
+        super().__init__(_L().sv_ngram_create(int(max_n), int(window)))
+
+    def begin_step(self):
+        _L().sv_ngram_begin_step(self._h)
+
+    def add(self, prompt_id: int, tokens):
+        t = _tok(tokens)
+        if _L().sv_ngram_add(self._h, int(prompt_id), t.ctypes.data, t.size) != 0:
+            raise ValueError("sv_ngram_add rejected its arguments")
+
+    def draft(self, prompt_id: int, context, k: int = 16) -> np.ndarray:
+        c = _tok(context)
+        out = np.empty(max(int(k), 1), np.int32)
+        n = _L().sv_ngram_draft(self._h, int(prompt_id), c.ctypes.data, c.size, int(k), out.ctypes.data)
+        if n < 0:
+            raise ValueError("sv_ngram_draft rejected its arguments")
+        return out[:n].copy()
+
+    def candidates(self, prompt_id: int, context, f: int) -> np.ndarray:
+        c = _tok(context)
+        out = np.empty(max(int(f), 1), np.int32)
+        n = _L().sv_ngram_candidates(self._h, int(prompt_id), c.ctypes.data, c.size, int(f), out.ctypes.data)
+        if n < 0:
+            raise ValueError("sv_ngram_candidates rejected its arguments")
+        return out[:n].copy()
+
+    @property
+    def rollouts(self) -> int:
+        return int(_L().sv_ngram_rollouts(self._h))
+
+    @property
+    def tokens(self) -> int:
+        return int(_L().sv_ngram_tokens(self._h))
+
+
+class SuffixDrafter(_Handle):
+    """Suffix drafter with frequency scoring (contexts up to ``max_depth``)."""
+    _destroy = "sv_suffix_destroy"
+
+    def __init__(self, max_depth: int = 8):
+        super().__init__(_L().sv_suffix_create(int(max_depth)))
+
+    def clear(self):
+        _L().sv_suffix_clear(self._h)
+
+    def append(self, problem_id: int, seq_id: int, tokens):
+        t = _tok(tokens)
+        if _L().sv_suffix_append(self._h, int(problem_id), int(seq_id), t.ctypes.data, t.size) != 0:
+            raise ValueError("sv_suffix_append rejected its arguments")
+
+    def draft(self, problem_id: int, context, k: int = 16) -> np.ndarray:
+        c = _tok(context)
+        out = np.empty(max(int(k), 1), np.int32)
+        n = _L().sv_suffix_draft(self._h, int(problem_id), c.ctypes.data, c.size, int(k), out.ctypes.data)
+        if n < 0:
+            raise ValueError("sv_suffix_draft rejected its arguments")
+        return out[:n].copy()
+
+    def candidates(self, problem_id: int, context, f: int) -> np.ndarray:
+        c = _tok(context)
+        out = np.empty(max(int(f), 1), np.int32)
+        n = _L().sv_suffix_candidates(self._h, int(problem_id), c.ctypes.data, c.size, int(f), out.ctypes.data)
+        if n < 0:
+            raise ValueError("sv_suffix_candidates rejected its arguments")
+        return out[:n].copy()
+
+
+class PrefetchBudget(_Handle):
+    """Fan-out prefetch budget over verification outcomes (j, rank of b)."""
+    _destroy = "sv_prefetch_destroy"
+
+    def __init__(self, k: int, fmax: int = 16, window: int = 256):
+        super().__init__(_L().sv_prefetch_create(int(k), int(fmax), int(window)))
+        self.k, self.fmax = int(k), int(fmax)
+
+    def observe(self, j: int, b_rank: int):
+        if _L().sv_prefetch_observe(self._h, int(j), int(b_rank)) != 0:
+            raise ValueError("sv_prefetch_observe rejected its arguments")
+
+    def estimates(self):
+        P = np.empty(self.k + 1, np.float64)
+        cov = np.empty((self.k + 1, self.fmax + 1), np.float64)
+        n = _L().sv_prefetch_estimates(self._h, P.ctypes.data, cov.ctypes.data)
+        return int(n), P, cov
+
+    def allocate(self, budget: int = 16):
+        f = np.empty(self.k + 1, np.int32)
+        cov = _L().sv_prefetch_allocate(self._h, int(budget), f.ctypes.data)
+        return f, float(cov)
+
+
+class DraftLengthController(_Handle):
+    """Adaptive draft length over ascending candidate lengths."""
+    _destroy = "sv_draft_len_destroy"
+
+    def __init__(self, lengths=(5, 7, 9, 11), up_frac: float = 0.7, down_frac: float = 0.4, patience: int = 2):
+        ls = _tok(lengths)
+        super().__init__(_L().sv_draft_len_create(ls.ctypes.data, ls.size, float(up_frac), float(down_frac),
+                                                  int(patience)))
+
+    @property
+    def current(self) -> int:
+        return int(_L().sv_draft_len_current(self._h))
+
+    def update(self, block_efficiency: float) -> int:
+        return int(_L().sv_draft_len_update(self._h, float(block_efficiency)))
+
+
+def block_efficiency(accept_len) -> float:
+    a = _tok(accept_len)
+    return float(_L().sv_block_efficiency(a.ctypes.data, a.size))
+
+
+def spec_switch(state: list, predicted_speedup: float, threshold: float = 1.05) -> int:
+    """``state`` is a one-element list holding the latch (0 at batch start)."""
+    s = ctypes.c_int32(int(state[0]))
+    r = _L().sv_spec_switch(ctypes.byref(s), float(predicted_speedup), float(threshold))
+    state[0] = int(s.value)
+    return int(r)
+
+
+def length_classes(predicted_len, budgets=(0, 8, 16)):
+    x = np.ascontiguousarray(np.asarray(predicted_len, np.float64).reshape(-1))
+    b = np.ascontiguousarray(np.asarray(budgets, np.int32).reshape(3))
+    cls = np.empty(x.size, np.int32)
+    bud = np.empty(x.size, np.int32)
+    if _L().sv_length_classes(x.ctypes.data, x.size, b.ctypes.data, cls.ctypes.data, bud.ctypes.data) != 0:
+        raise ValueError("sv_length_classes rejected its arguments")
+    return cls, bud
+
+
+def interleave_ranks(predicted_len, world_size: int):
+    x = np.ascontiguousarray(np.asarray(predicted_len, np.float64).reshape(-1))
+    r = np.empty(x.size, np.int32)
+    if _L().sv_interleave_ranks(x.ctypes.data, x.size, int(world_size), r.ctypes.data) != 0:
+        raise ValueError("sv_interleave_ranks rejected its arguments")
+    return r

@@ -1,0 +1,339 @@
+"""Host-side components (include/sv_host.h), CPU only.
+
+Pins tie the plain-Python oracle (oracle/host_policy.py) to what the pages
+state; parity tests run the C++ implementation and the oracle on the same
+seeded synthetic token streams and outcomes and require identical results.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from speculative_decoding_verification_92_b200 import host
+from oracle import host_policy as ho
+
+
+# ---------------------------------------------------------------------------
+# pins: n-gram drafter ("AI 开始抄自己的作业——而且抄得理直气壮",
+# section "📓 NgramRL：每道题配一本活页草稿本")
+
+def test_pin_ngram_page_example():
+    """A generation ending in "so the final answer is" is drafted with the
+    continuation the prompt's earlier rollout wrote after that prefix."""
+    SO, FINAL, ANSWER, IS, N42, COMMA, BECAUSE = 101, 102, 103, 104, 42, 7, 105
+    tail = [N42, COMMA, BECAUSE] + list(range(200, 220))
+    rollout = [1, 2, 3, SO, FINAL, ANSWER, IS] + tail
+    for drafter in (ho.NgramOracle(6, 4), host.NgramDrafter(6, 4)):
+        drafter.begin_step()
+        drafter.add(7, rollout)
+        got = list(drafter.draft(7, [9, 9, SO, FINAL, ANSWER, IS], 16))
+        assert got == tail[:16]
+        assert list(drafter.draft(8, [SO, FINAL, ANSWER, IS], 16)) == []   # per-prompt tables
+
+
+def test_pin_ngram_window_and_recency():
+    for d in (ho.NgramOracle(6, 4), host.NgramDrafter(6, 4)):
+        d.begin_step()                       # step 0
+        d.add(1, [5, 6, 7, 8])
+        for _ in range(3):                   # steps 1..3: still within W = 4
+            d.begin_step()
+            assert list(d.draft(1, [5, 6], 4)) == [7, 8]
+        d.add(1, [5, 6, 9, 9])               # a newer rollout wins the same match
+        assert list(d.draft(1, [5, 6], 4)) == [9, 9]
+        d.begin_step()                       # step 4: step 0 falls out of the window
+        assert list(d.draft(1, [5, 6], 4)) == [9, 9]
+        assert list(d.draft(1, [6, 7], 4)) == []
+        for _ in range(4):
+            d.begin_step()
+        assert list(d.draft(1, [5, 6], 4)) == []
+
+
+def test_pin_ngram_longest_match_capped_at_n():
+    # the 7-gram 1..7 continues with 50 in the old rollout; the newer rollout
+    # shares only the 6-gram 2..7 and continues with 60
+    old, new = [1, 2, 3, 4, 5, 6, 7, 50], [9, 2, 3, 4, 5, 6, 7, 60]
+    ctx = [1, 2, 3, 4, 5, 6, 7]
+    for max_n, want in ((6, 60), (7, 50)):
+        for d in (ho.NgramOracle(max_n, 4), host.NgramDrafter(max_n, 4)):
+            d.begin_step()
+            d.add(0, old)
+            d.add(0, new)
+            assert list(d.draft(0, ctx, 1)) == [want], (max_n, type(d).__name__)
+
+
+# pins: suffix drafter (Together AI blog, "Adaptive suffix tree drafter")
+
+def test_pin_suffix_frequency_and_immediate_insertion():
+    A, B, C, D = 1, 2, 3, 4
+    for s in (ho.SuffixOracle(4), host.SuffixDrafter(4)):
+        for i in range(3):
+            s.append(0, i, [A, B, C])
+        s.append(0, 3, [A, B, D])
+        assert list(s.draft(0, [A, B], 1)) == [C]
+        assert list(s.candidates(0, [A, B], 4)) == [C, D]
+        s.append(0, 4, [A, B, D, A, B, D, A, B, D])   # verified tokens count at once
+        assert list(s.draft(0, [A, B], 1)) == [D]
+        s.clear()
+        assert list(s.draft(0, [A, B], 1)) == []
+
+
+# pins: fan-out prefetch ("🚰 真正的瓶颈不在算法，在流水线")
+
+def test_pin_prefetch_all_accepted_branch_needs_one_candidate():
+    """When the all-accepted branch's top candidate is right 90% of the time
+    and the next ones add nothing, it gets exactly one of N = 16 slots."""
+    k, fmax = 4, 16
+    rng = np.random.default_rng(3)
+    obs = []
+    for t in range(400):
+        j = k if t % 2 == 0 else int(rng.integers(0, k))
+        if j == k:
+            r = 0 if rng.random() < 0.9 else -1
+        else:
+            r = int(min(rng.geometric(0.35) - 1, fmax))
+            r = -1 if r >= fmax else r
+        obs.append((j, r))
+    f, _ = ho.prefetch_allocate(obs, k, fmax, 400, 16)
+    assert f[k] == 1 and sum(f) == 16
+    p = host.PrefetchBudget(k, fmax, 400)
+    for j, r in obs:
+        p.observe(j, r)
+    fc, _ = p.allocate(16)
+    assert list(fc) == f
+
+
+def test_pin_prefetch_greedy_is_optimal_for_concave_profiles():
+    """With coverage increments that never grow (the drafter ranks well),
+    the greedy allocation reaches the best expected coverage of all
+    allocations of the budget (exhaustive search)."""
+    rng = np.random.default_rng(5)
+    for trial in range(30):
+        k, fmax, budget = 2, 4, int(rng.integers(1, 7))
+        obs = []
+        for _ in range(60):
+            j = int(rng.integers(0, k + 1))
+            r = int(min(rng.geometric(0.5) - 1, fmax))     # decreasing rank probabilities
+            obs.append((j, -1 if r >= fmax else r))
+        n, P, cov = ho.prefetch_estimates(obs, k, fmax, 60)
+        for j in range(k + 1):
+            inc = np.diff(cov[j])
+            if not np.all(inc[1:] <= inc[:-1] + 1e-12):
+                break
+        else:
+            f, total = ho.prefetch_allocate(obs, k, fmax, 60, budget)
+            best = max(ho.expected_coverage(P, cov, list(a))
+                       for a in itertools.product(range(fmax + 1), repeat=k + 1) if sum(a) <= budget)
+            assert abs(total - best) < 1e-12 and abs(ho.expected_coverage(P, cov, f) - best) < 1e-12
+
+
+def test_pin_prefetch_window_is_causal():
+    k, fmax = 3, 4
+    early = [(0, -1)] * 50
+    late = [(3, 0)] * 20
+    n, P, cov = ho.prefetch_estimates(early + late, k, fmax, 20)
+    assert n == 20 and P == [0, 0, 0, 1.0] and cov[3][1] == 1.0
+    p = host.PrefetchBudget(k, fmax, 20)
+    for j, r in early + late:
+        p.observe(j, r)
+    n2, P2, cov2 = p.estimates()
+    assert n2 == 20 and np.allclose(P2, P) and np.allclose(cov2, cov)
+    f, total = p.allocate(16)
+    assert list(f) == [0, 0, 0, 1] and total == 1.0
+    assert list(host.PrefetchBudget(k, fmax, 20).allocate(16)[0]) == [0, 0, 0, 0]   # empty window
+
+
+# pins: draft length and switch (EfficientRollout article, sections
+# "四、自适应草稿长度" and "三、聪明的开关")
+
+def block_eff(alpha, k):
+    """Block efficiency of i.i.d. per-token acceptance alpha with draft length k."""
+    return (1 - alpha ** (k + 1)) / (1 - alpha)
+
+
+def test_pin_draft_length_rises_5_7_9_11_as_acceptance_grows():
+    lengths = [5, 7, 9, 11]
+    alphas = np.linspace(0.70, 0.97, 40)
+    c = host.DraftLengthController(lengths)
+    used = []
+    for a in alphas:
+        used.append(c.current)
+        c.update(block_eff(a, c.current))
+    assert used[0] == 5 and c.current == 11
+    assert [x for i, x in enumerate(used) if i == 0 or x != used[i - 1]] == lengths   # 5 -> 7 -> 9 -> 11
+    o_used, o_last = ho.draft_length_trajectory(lengths, [block_eff(a, u) for a, u in zip(alphas, used)])
+    assert o_used == used and o_last == c.current
+
+
+def test_pin_draft_length_ignores_one_step_blips():
+    c = host.DraftLengthController([5, 7, 9, 11])
+    for tau in (5.5, 2.0, 5.5, 2.0, 5.5):        # never two high steps in a row
+        assert c.update(tau) == 5
+    assert c.update(5.5) == 7                    # two in a row: up
+    assert c.update(1.0) == 7 and c.update(1.0) == 5   # two low steps: down
+    assert c.update(float("nan")) == 5
+
+
+def test_pin_block_efficiency_and_switch():
+    assert host.block_efficiency([0, 3, 8, -1, -2]) == pytest.approx((1 + 4 + 9) / 3)
+    assert math.isnan(host.block_efficiency([-1, -2]))
+    preds = [0.9, 1.02, 1.051, 0.8, 1.2]
+    want = ho.spec_switch(preds)
+    assert want == [0, 0, 1, 1, 1]
+    state = [0]
+    assert [host.spec_switch(state, s) for s in preds] == want
+
+
+# pins: budgets (Together AI blog, "Length-aware scheduling")
+
+def test_pin_length_classes_and_rank_interleave():
+    pred = [100, 900, 50, 400, 800, 30, 600, 200, 700]
+    cls, bud = host.length_classes(pred, (0, 8, 16))
+    assert sorted(np.array(pred)[cls == 2]) == [700, 800, 900]
+    assert sorted(np.array(pred)[cls == 0]) == [30, 50, 100]
+    assert set(bud[cls == 0]) == {0} and set(bud[cls == 2]) == {16}
+    ranks = host.interleave_ranks([1000] * 8 + [10] * 8, 2)
+    assert list(np.bincount(ranks[:8])) == [4, 4] and list(np.bincount(ranks[8:])) == [4, 4]
+
+
+# ---------------------------------------------------------------------------
+# parity: C++ against the oracle on seeded synthetic streams
+
+def markov_stream(rng, n, vocab, stick=0.8):
+    """Tokens from a sticky random chain (so n-grams repeat)."""
+    nxt = rng.integers(0, vocab, size=vocab)
+    out = [int(rng.integers(0, vocab))]
+    for _ in range(n - 1):
+        out.append(int(nxt[out[-1]]) if rng.random() < stick else int(rng.integers(0, vocab)))
+    return out
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_ngram_parity(seed):
+    rng = np.random.default_rng(100 + seed)
+    max_n, window = int(rng.integers(1, 7)), int(rng.integers(1, 5))
+    o, c = ho.NgramOracle(max_n, window), host.NgramDrafter(max_n, window)
+    for step in range(7):
+        o.begin_step()
+        c.begin_step()
+        for _ in range(int(rng.integers(0, 6))):
+            pid = int(rng.integers(0, 3))
+            toks = markov_stream(rng, int(rng.integers(0, 60)), 12)
+            o.add(pid, toks)
+            c.add(pid, toks)
+        for _ in range(40):
+            pid = int(rng.integers(0, 4))
+            ctx = markov_stream(rng, int(rng.integers(0, 12)), 12)
+            k, f = int(rng.integers(0, 20)), int(rng.integers(0, 6))
+            assert list(c.draft(pid, ctx, k)) == o.draft(pid, ctx, k)
+            assert list(c.candidates(pid, ctx, f)) == o.candidates(pid, ctx, f)
+        assert c.rollouts == sum(len(v) for v in o.rollouts.values())
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_suffix_parity(seed):
+    rng = np.random.default_rng(200 + seed)
+    depth = int(rng.integers(1, 9))
+    o, c = ho.SuffixOracle(depth), host.SuffixDrafter(depth)
+    for _ in range(60):
+        pid, sid = int(rng.integers(0, 3)), int(rng.integers(0, 4))
+        toks = markov_stream(rng, int(rng.integers(0, 25)), 10)
+        o.append(pid, sid, toks)
+        c.append(pid, sid, toks)
+        ctx = markov_stream(rng, int(rng.integers(0, 10)), 10)
+        k, f = int(rng.integers(0, 20)), int(rng.integers(0, 6))
+        assert list(c.draft(pid, ctx, k)) == o.draft(pid, ctx, k)
+        assert list(c.candidates(pid, ctx, f)) == o.candidates(pid, ctx, f)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_prefetch_parity(seed):
+    rng = np.random.default_rng(300 + seed)
+    k, fmax, window = int(rng.integers(0, 8)), int(rng.integers(1, 17)), int(rng.integers(1, 80))
+    p, obs = host.PrefetchBudget(k, fmax, window), []
+    for t in range(150):
+        j, r = int(rng.integers(0, k + 1)), int(rng.integers(-1, fmax + 3))
+        p.observe(j, r)
+        obs.append((j, -1 if r >= fmax else r))
+        if t % 7 == 0:
+            budget = int(rng.integers(0, 20))
+            f, total = p.allocate(budget)
+            fo, to = ho.prefetch_allocate(obs, k, fmax, window, budget)
+            assert list(f) == fo and abs(total - to) < 1e-12
+            n, P, cov = p.estimates()
+            no, Po, covo = ho.prefetch_estimates(obs, k, fmax, window)
+            assert n == no and np.allclose(P, Po, rtol=0, atol=1e-15) and np.allclose(cov, covo, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_controller_and_budget_parity(seed):
+    rng = np.random.default_rng(400 + seed)
+    lengths = sorted(set(int(x) for x in rng.integers(1, 20, size=int(rng.integers(1, 6)))))
+    up, down = sorted(rng.uniform(0.1, 0.95, 2))[::-1]
+    patience = int(rng.integers(1, 4))
+    c = host.DraftLengthController(lengths, up, down, patience)
+    used, taus = [], []
+    for _ in range(60):
+        used.append(c.current)
+        tau = float(rng.uniform(0.5, c.current + 1))
+        taus.append(tau)
+        c.update(tau)
+    o_used, o_last = ho.draft_length_trajectory(lengths, taus, up, down, patience)
+    assert used == o_used and c.current == o_last
+    for n in (0, 1, 2, 5, 17):
+        pred = rng.integers(0, 6, size=n).astype(float)      # many ties
+        cls, bud = host.length_classes(pred, (0, 4, 12))
+        ocls, obud = ho.length_classes(list(pred), (0, 4, 12))
+        assert list(cls) == ocls and list(bud) == obud
+        for world in (1, 2, 3, 8):
+            assert list(host.interleave_ranks(pred, world)) == ho.interleave_ranks(list(pred), world)
+
+
+def test_bad_arguments_are_rejected():
+    with pytest.raises(ValueError):
+        host.NgramDrafter(0, 4)
+    with pytest.raises(ValueError):
+        host.SuffixDrafter(0)
+    with pytest.raises(ValueError):
+        host.PrefetchBudget(-1)
+    with pytest.raises(ValueError):
+        host.DraftLengthController([5, 5])
+    with pytest.raises(ValueError):
+        host.DraftLengthController([5, 7], up_frac=0.3, down_frac=0.5)
+    p = host.PrefetchBudget(3, 4, 8)
+    with pytest.raises(ValueError):
+        p.observe(4, 0)
+    with pytest.raises(ValueError):
+        host.length_classes([1.0, float("nan")])
+
+
+# ---------------------------------------------------------------------------
+# end to end on synthetic rollouts: drafts from the table, prefix-match
+# verification against the rollout the policy actually writes
+
+def test_ngram_speculation_on_repeating_rollouts():
+    """The more the same prompt's rollouts repeat across steps (the page
+    measures 50% early, 81% mid, 100% late), the more drafted tokens each
+    verification accepts; at full repetition every draft of 16 is accepted."""
+    rng = np.random.default_rng(9)
+    base = [int(x) for x in rng.integers(0, 5000, 400)]   # its 2-grams do not repeat
+    assert len({tuple(base[i:i + 2]) for i in range(399)}) == 399
+
+    def accepted_per_cycle(copy_prob):
+        d = host.NgramDrafter(6, 4)
+        d.begin_step()
+        d.add(0, base)
+        target = [t if rng.random() < copy_prob else int(rng.integers(0, 5000)) for t in base]
+        pos, acc, cycles = 8, 0, 0
+        while pos < len(target) - 17:
+            draft = d.draft(0, target[:pos], 16)
+            j = 0
+            while j < len(draft) and draft[j] == target[pos + j]:
+                j += 1
+            acc += j
+            cycles += 1
+            pos += j + 1
+        return acc / cycles
+
+    rates = [accepted_per_cycle(p) for p in (0.5, 0.81, 1.0)]
+    assert rates[0] < rates[1] < rates[2] and rates[2] == 16.0
