@@ -76,6 +76,8 @@ def parse_args():
     ap.add_argument("--greedy", action="store_true", help="time the greedy (prefix-match) form instead")
     ap.add_argument("--event-every", type=int, default=16,
                     help="bracket the row-statistics kernel with events on every N-th timed step")
+    ap.add_argument("--host", action="store_true",
+                    help="time the host-side drafters and prefetch budget instead (CPU only)")
     return ap.parse_args()
 
 
@@ -302,8 +304,79 @@ def run_reference(args):
     return 0
 
 
+def run_host(args):
+    """Host-side components on a synthetic RL rollout history: 64 prompts x 5
+    rollouts per step over W = 4 steps (the NgramRL setup), each rollout a
+    copy of the prompt's previous one with 10% of its tokens replaced.
+    Times draft lookups (k = 16) and ranked candidates (f = 16) of the C++
+    n-gram and suffix drafters, and the prefetch allocation; the plain-Python
+    oracle is timed on a bounded sample of the same lookups."""
+    import numpy as np
+
+    from speculative_decoding_verification_92_b200 import host
+    from oracle import host_policy as ho
+
+    rng = np.random.default_rng(92)
+    P, R, T, W, V = 64, 5, 1024, 4, 151936
+    base = [rng.integers(0, V, T).astype(np.int32) for _ in range(P)]
+    ng, sx, o_ng = host.NgramDrafter(6, W), host.SuffixDrafter(8), ho.NgramOracle(6, W)
+    t0 = time.perf_counter()
+    for step in range(W):
+        ng.begin_step()
+        o_ng.begin_step()
+        for p in range(P):
+            for r in range(R):
+                roll = base[p].copy()
+                m = rng.random(T) < 0.1
+                roll[m] = rng.integers(0, V, int(m.sum()))
+                ng.add(p, roll)
+                o_ng.add(p, roll)
+                if step == W - 1:
+                    sx.append(p, r, roll)
+                base[p] = roll
+    build_s = time.perf_counter() - t0
+    queries = [(int(rng.integers(0, P)), int(rng.integers(8, T))) for _ in range(20000)]
+    ctxs = [base[p][max(0, q - 32):q] for p, q in queries]
+
+    def rate(fn, items, budget_s):
+        n, t0 = 0, time.perf_counter()
+        for it in items:
+            fn(*it)
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        return n / (time.perf_counter() - t0), n
+
+    items = [(p, c) for (p, _), c in zip(queries, ctxs)]
+    ng_rate, _ = rate(lambda p, c: ng.draft(p, c, 16), items, 5.0)
+    ng_cand, _ = rate(lambda p, c: ng.candidates(p, c, 16), items, 5.0)
+    sx_rate, _ = rate(lambda p, c: sx.draft(p, c, 16), items, 5.0)
+    o_rate, o_n = rate(lambda p, c: o_ng.draft(p, list(c), 16), items, args.cpu_seconds)
+    pf = host.PrefetchBudget(16, 16, 256)
+    for _ in range(256):
+        pf.observe(int(rng.integers(0, 17)), int(rng.integers(-1, 16)))
+    pf_rate, _ = rate(lambda b: pf.allocate(b), [(16,)] * 200000, 2.0)
+    accepted = []
+    for p, c in items[:2000]:
+        d = ng.draft(p, c, 16)
+        accepted.append(len(d))
+    line = {
+        "metric": "host n-gram draft lookups/s (k=16), 1 core", "value": ng_rate, "unit": "lookups/s",
+        "data": "synthetic", "config": {"workload": f"{P} prompts x {R} rollouts x {T} tokens, W={W} steps, "
+                                                    "10% token changes per rollout", "max_n": 6, "k": 16},
+        "ngram_candidates_per_s": ng_cand, "suffix_draft_per_s": sx_rate, "prefetch_allocations_per_s": pf_rate,
+        "table_build_s": build_s, "retained_tokens": ng.tokens, "mean_draft_len": float(np.mean(accepted)),
+        "cpu_baseline": {"value": o_rate, "unit": "lookups/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{o_n} n-gram draft lookups with the plain-Python oracle"},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.host:
+        return run_host(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours_impl(args)
