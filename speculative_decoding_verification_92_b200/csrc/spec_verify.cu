@@ -18,7 +18,6 @@ namespace {
 
 constexpr int kTmaConsumerWarps = SV_TMA_CONSUMER_WARPS;
 constexpr int kTmaStages = SV_TMA_STAGES;
-constexpr int kTmaCtasPerSm = SV_TMA_CTAS_PER_SM;
 constexpr int kLdgThreads = 256;
 // Draw-kernel grid: about SV_DRAW_WAVES waves of kDrawCtasPerSm CTAs per SM.
 #ifndef SV_DRAW_WAVES
@@ -143,7 +142,14 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
             auto k = row_stats_tma_kernel<T, kGreedy, kTmaConsumerWarps, kTmaStages>;
             const size_t smem = TmaSmem<kTmaConsumerWarps, kTmaStages>::bytes(prm.nB);
             if ((e = allow_smem(k, smem)) != cudaSuccess) return e;
-            const int64_t cap = int64_t(dev.sm_count) * kTmaCtasPerSm;
+            // one wave of resident CTAs (a long request list can make the
+            // row prefix in shared memory lower the occupancy)
+            int per_sm = 0;
+            if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, (kTmaConsumerWarps + 1) * 32, smem)) !=
+                cudaSuccess)
+                return e;
+            per_sm = per_sm < 1 ? 1 : (per_sm > TmaCtasPerSm<T>::value ? TmaCtasPerSm<T>::value : per_sm);
+            const int64_t cap = int64_t(dev.sm_count) * per_sm;
             const int64_t grid = items_upper < cap ? items_upper : cap;
             cfg.gridDim = dim3(static_cast<unsigned>(grid));
             cfg.blockDim = dim3((kTmaConsumerWarps + 1) * 32);
@@ -289,7 +295,10 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     dp.out_weights = a.out_weights;
     dp.decay = a.decay;
     dp.rows_aligned = rows_aligned ? 1 : 0;
-    dp.fast_draw = (rows_aligned && !greedy && !a.stats_only && int64_t(plan.CE) * plan.es <= kMaxChunkBytesFast) ? 1 : 0;
+    // the ring pass needs whole pieces per chunk and at most kMaxSegsPerChunk segments
+    const int64_t chunk_bytes = int64_t(plan.CE) * plan.es;
+    dp.fast_draw = (rows_aligned && !greedy && !a.stats_only && chunk_bytes <= kMaxChunkBytesFast &&
+                    chunk_bytes % (int64_t(kPieceVecs) * 16) == 0) ? 1 : 0;
     {
         // fewest chunks per CTA that fit the batch in about SV_DRAW_WAVES
         // waves, then spread evenly: C2 = ceil(C / r) CTAs of ceil(C / C2) chunks

@@ -32,10 +32,16 @@
 #define SV_TMA_CONSUMER_WARPS 4
 #endif
 #ifndef SV_TMA_STAGES
-#define SV_TMA_STAGES 3
+#define SV_TMA_STAGES 2
 #endif
-#ifndef SV_TMA_CTAS_PER_SM
-#define SV_TMA_CTAS_PER_SM 4
+// Resident CTAs per SM the bulk-copy variant is built for, per logit type:
+// bf16 spends twice the exps per byte of fp32, so it wants more consumer warps
+// in flight (6 x 4 on B200); fp32 does best at 5 x 4.
+#ifndef SV_TMA_CTAS_PER_SM_BF16
+#define SV_TMA_CTAS_PER_SM_BF16 6
+#endif
+#ifndef SV_TMA_CTAS_PER_SM_F32
+#define SV_TMA_CTAS_PER_SM_F32 5
 #endif
 // 16-byte vectors per thread in flight in the vector-load variant.
 #ifndef SV_LDG_UNROLL
@@ -348,6 +354,11 @@ __device__ __forceinline__ void fold_vector(Acc<kGreedy>& acc, const uint4& w, i
 
 constexpr int kStageBytes = SV_STAGE_BYTES;
 
+template <typename T>
+struct TmaCtasPerSm {
+    static constexpr int value = Logit<T>::kSize == 2 ? SV_TMA_CTAS_PER_SM_BF16 : SV_TMA_CTAS_PER_SM_F32;
+};
+
 struct StageMeta {
     const unsigned char* tail;  // first ragged-tail element (row's last chunk), or null
     int64_t partial_idx;
@@ -368,7 +379,7 @@ struct TmaSmem {
 };
 
 template <typename T, bool kGreedy, int kConsumerWarps, int kStages>
-__global__ void __launch_bounds__((kConsumerWarps + 1) * 32, SV_TMA_CTAS_PER_SM)
+__global__ void __launch_bounds__((kConsumerWarps + 1) * 32, TmaCtasPerSm<T>::value)
 row_stats_tma_kernel(const StatsParams p) {
     constexpr int kConsumers = kConsumerWarps * 32;
     constexpr int kThreads = kConsumers + 32;
