@@ -113,7 +113,10 @@ typedef enum {
     SV_STATS_AUTO = 0,
     SV_STATS_TMA = 1,    /* cp.async.bulk + mbarrier ring; needs 16-byte aligned rows */
     SV_STATS_VEC16 = 2,  /* 16-byte vector loads; needs 16-byte aligned rows */
-    SV_STATS_SCALAR = 3  /* element loads; any alignment */
+    SV_STATS_SCALAR = 3, /* element loads; any alignment */
+    SV_STATS_FUSED = 4   /* sampling only: the whole step in one persistent launch
+                            (statistics, scan and draw through one bulk-copy ring);
+                            needs 16-byte aligned rows, B <= 4096 */
 } sv_stats_kernel;
 
 typedef struct {

@@ -43,6 +43,7 @@ class StatsKernel(enum.IntEnum):
     TMA = 1
     VEC16 = 2
     SCALAR = 3
+    FUSED = 4    # sampling only: statistics, scan and draw in one persistent launch
 
 
 class SpecVerifyError(RuntimeError):

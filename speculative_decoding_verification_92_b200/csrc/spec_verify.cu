@@ -12,6 +12,7 @@
 #include "sv_common.cuh"
 #include "sv_row_stats.cuh"
 #include "sv_verify_draw.cuh"
+#include "sv_fused.cuh"
 
 namespace sv {
 namespace {
@@ -117,9 +118,20 @@ bool shape_ok(const sv_shape* s, sv_status* why) {
     return true;
 }
 
+// Segments of 32 vectors in one chunk (the draw's finest sums).
+int nseg_max_of(const Plan& p) {
+    const int vecs = (p.CE * p.es + 15) / 16;
+    return (vecs + kSegVecs - 1) / kSegVecs;
+}
+
+// The two-kernel path uses the first part (C partials per row); the fused
+// path lays out W partials per chunk plus its counters, queue and sums.
 size_t workspace_bytes_for(const sv_shape& s, const Plan& p) {
     const size_t n = size_t(s.B) * size_t(2 * s.k_max + 1) * size_t(p.C) * sizeof(float2);
-    return (n + 255) & ~size_t(255);
+    const size_t two_kernel = (n + 255) & ~size_t(255);
+    const size_t fused =
+        fused_layout(s.B, s.k_max, p.C, kTmaConsumerWarps, nseg_max_of(p), p.CE * p.es / kPieceBytes).total;
+    return two_kernel > fused ? two_kernel : fused;
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -312,6 +324,78 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     return e == cudaSuccess ? SV_OK : SV_ECUDA;
 }
 
+// Whether the one-launch path can run this call.
+bool fused_ok(const Call& a, const Plan& plan, bool rows_aligned) {
+    const sv_shape& s = *a.shape;
+    const int64_t chunk_bytes = int64_t(plan.CE) * plan.es;
+    return !a.greedy && !a.stats_only && rows_aligned && s.B <= kMaxRequestsPerLaunch && s.k_max >= 0 &&
+           chunk_bytes <= kMaxChunkBytesFast && chunk_bytes % kPieceBytes == 0 && plan.C <= kMaxChunks;
+}
+
+template <typename T>
+sv_status run_fused(const Call& a, const Plan& plan, const DeviceInfo& dev) {
+    const sv_shape& s = *a.shape;
+    const int nseg_max = nseg_max_of(plan);
+    const int P = plan.CE * plan.es / kPieceBytes;   // draw pieces per chunk
+    const FusedLayout l = fused_layout(s.B, s.k_max, plan.C, kTmaConsumerWarps, nseg_max, P);
+    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+    FusedParams fp{};
+    fp.target = static_cast<const unsigned char*>(a.target);
+    fp.draft = static_cast<const unsigned char*>(a.draft);
+    fp.tokens = a.tokens;
+    fp.lens = a.lens;
+    fp.uniforms = a.uniforms;
+    fp.out_len = a.out_len;
+    fp.out_tokens = a.out_tokens;
+    fp.partials = reinterpret_cast<float2*>(ws + l.partials);
+    fp.state = reinterpret_cast<FusedState*>(ws + l.state);
+    fp.done_items = reinterpret_cast<int32_t*>(ws + l.done_items);
+    fp.draw_done = reinterpret_cast<int32_t*>(ws + l.draw_done);
+    fp.final_flag = reinterpret_cast<int32_t*>(ws + l.final_flag);
+    fp.mbox_ready = reinterpret_cast<int32_t*>(ws + l.mbox_ready);
+    fp.mbox_task = reinterpret_cast<int32_t*>(ws + l.mbox_task);
+    fp.req = reinterpret_cast<FusedReq*>(ws + l.req);
+    fp.segs = reinterpret_cast<float*>(ws + l.segs);
+    fp.piece_tot = reinterpret_cast<float*>(ws + l.piece_tot);
+    fp.P = P;
+    fp.B = s.B;
+    fp.k_max = s.k_max;
+    fp.V = s.V;
+    fp.row_stride = plan.stride;
+    fp.C = plan.C;
+    fp.CE = plan.CE;
+    fp.nseg_max = nseg_max;
+    fp.scale = static_cast<float>(kLog2e / static_cast<double>(a.temperature));
+    const int tmo = a.opts ? a.opts->wait_timeout_us : 0;
+    fp.timeout_ns = tmo > 0 ? uint64_t(tmo) * 1000ull : kDefaultTimeoutNs;
+
+    cudaError_t e = cudaMemsetAsync(ws + l.zero_begin, 0, l.zero_end - l.zero_begin, a.stream);
+    if (e != cudaSuccess) return SV_ECUDA;
+    auto k = verify_fused_kernel<T, kTmaConsumerWarps, kTmaStages>;
+    const size_t smem = FusedSmem<kTmaConsumerWarps, kTmaStages>::bytes(s.B, nseg_max);
+    if ((e = allow_smem(k, smem)) != cudaSuccess) return SV_ECUDA;
+    constexpr int kThreadsF = (kTmaConsumerWarps + 1) * 32;
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreadsF, smem)) != cudaSuccess)
+        return SV_ECUDA;
+    per_sm = per_sm < 1 ? 1 : (per_sm > TmaCtasPerSm<T>::value ? TmaCtasPerSm<T>::value : per_sm);
+    const int rows_max = a.draft ? 2 * s.k_max + 1 : s.k_max + 1;
+    const int64_t work = int64_t(s.B) * rows_max * plan.C;
+    int64_t cap = int64_t(dev.sm_count) * per_sm;
+    cap = cap < kMaxFusedGrid ? cap : kMaxFusedGrid;
+    const int64_t grid = work < cap ? (work < 1 ? 1 : work) : cap;
+    fp.mbox_slots = static_cast<int>((int64_t(s.B) * plan.C * P + grid - 1) / grid + 1);
+    if (a.opts && a.opts->event_stats_begin)
+        if (cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_begin), a.stream) != cudaSuccess)
+            return SV_ECUDA;
+    k<<<dim3(static_cast<unsigned>(grid)), dim3(kThreadsF), smem, a.stream>>>(fp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return SV_ECUDA;
+    if (a.opts && a.opts->event_stats_end)
+        if (cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_end), a.stream) != cudaSuccess)
+            return SV_ECUDA;
+    return SV_OK;
+}
+
 sv_status run(const Call& a) {
     sv_status why = SV_OK;
     if (!shape_ok(a.shape, &why)) return why;
@@ -319,7 +403,7 @@ sv_status run(const Call& a) {
     if (a.opts) {
         for (int i = 0; i < 8; ++i)
             if (a.opts->reserved[i] != 0) return SV_EINVAL;
-        if (a.opts->stats_kernel < SV_STATS_AUTO || a.opts->stats_kernel > SV_STATS_SCALAR) return SV_EINVAL;
+        if (a.opts->stats_kernel < SV_STATS_AUTO || a.opts->stats_kernel > SV_STATS_FUSED) return SV_EINVAL;
         if (a.opts->wait_timeout_us < 0) return SV_EINVAL;
     }
     if (s.B == 0) return SV_OK;
@@ -354,6 +438,10 @@ sv_status run(const Call& a) {
     int variant = a.opts ? a.opts->stats_kernel : SV_STATS_AUTO;
     if (variant == SV_STATS_AUTO) variant = rows_aligned ? SV_STATS_TMA : SV_STATS_SCALAR;
     if ((variant == SV_STATS_TMA || variant == SV_STATS_VEC16) && !rows_aligned) return SV_EINVAL;
+    if (variant == SV_STATS_FUSED) {
+        if (!fused_ok(a, plan, rows_aligned)) return SV_EINVAL;
+        return s.dtype == SV_BF16 ? run_fused<bf16_bits>(a, plan, *dev) : run_fused<float>(a, plan, *dev);
+    }
 
     return s.dtype == SV_BF16 ? run_typed<bf16_bits>(a, plan, *dev, variant, rows_aligned)
                               : run_typed<float>(a, plan, *dev, variant, rows_aligned);

@@ -49,12 +49,26 @@ def plan_chunks(V, es):
     return -(-V // ce), ce
 
 
+def a256(n):
+    return (n + 255) // 256 * 256
+
+
+def fused_bytes(B, k, C, CE, es, W=4):
+    """The one-launch layout: W partials per chunk, counters, task queue,
+    per-request records (48 B) and one sum per 32-vector segment."""
+    nseg = -(-(CE * es // 16) // 32)
+    P = CE * es // 8192               # draw pieces (one 8 KiB ring stage per row) per chunk
+    mbox = B * C * P + 2 * 1024       # per-CTA task mailboxes
+    return (a256(8 * B * (2 * k + 1) * C * W) + a256(32) + 3 * a256(4 * B) + a256(4 * mbox)
+            + a256(4 * mbox) + a256(48 * B) + a256(4 * B * C * nseg) + a256(4 * B * C * P * W))
+
+
 @pytest.mark.parametrize("B,k,V,dt", [(64, 8, 151936, sv.BF16), (256, 12, 128256, sv.F32),
                                       (4, 4, 1000, sv.F32), (3, 0, 5, sv.BF16), (0, 3, 100, sv.F32)])
 def test_workspace_bytes(B, k, V, dt):
-    C, _ = plan_chunks(V, 2 if dt == sv.BF16 else 4)
-    want = B * (2 * k + 1) * C * 8
-    want = (want + 255) // 256 * 256
+    es = 2 if dt == sv.BF16 else 4
+    C, CE = plan_chunks(V, es)
+    want = max(a256(B * (2 * k + 1) * C * 8), fused_bytes(B, k, C, CE, es))
     assert sv.workspace_bytes(B, k, V, dt) == want
 
 
