@@ -63,7 +63,8 @@
  * out-of-bounds access: a request whose draft_lens entry is outside
  * [0, k_max] or whose first L_b drafted ids are outside [0, V) gets
  * out_accept_len = -1 and out_tokens all -1; a request whose statistics were
- * lost to a device-side wait timeout gets out_accept_len = -2.  NaN or +inf
+ * lost to a device-side wait timeout gets out_accept_len = -2 (tests make a
+ * wait run out through sv_options.lost_copy_request).  NaN or +inf
  * logits in rows that are read give unspecified (but in-bounds) results.
  */
 #ifndef SPEC_VERIFY_H
@@ -124,7 +125,16 @@ typedef struct {
     int32_t wait_timeout_us;   /* bound on each device-side barrier wait; 0 = 2 s */
     void *event_stats_begin;   /* cudaEvent_t recorded just before the row-statistics kernel, or NULL */
     void *event_stats_end;     /* cudaEvent_t recorded just after it, or NULL */
-    int32_t reserved[8];       /* must be zero */
+    /* Fault injection for tests of the wait bound; 0 = off.  A value r > 0
+     * names request b = r - 1 (0 <= b < B): the bulk-copy statistics kernel
+     * then never issues the copy of the first stage of b's target row 0,
+     * chunk 0.  The wait on that stage runs out after wait_timeout_us, and b
+     * gets out_accept_len = -2 (so may other requests whose statistics fell
+     * to the same CTA after it); the call itself still returns SV_OK and the
+     * context stays usable.  Needs the bulk-copy kernel (SV_STATS_TMA, or
+     * AUTO on aligned rows): with any other kernel, SV_EUNSUPPORTED. */
+    int32_t lost_copy_request;
+    int32_t reserved[7];       /* must be zero */
 } sv_options;
 
 /* Bytes of device workspace spec_verify / spec_verify_stats need for this

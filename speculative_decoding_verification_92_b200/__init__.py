@@ -60,7 +60,7 @@ class _Shape(ctypes.Structure):
 class _Options(ctypes.Structure):
     _fields_ = [("stats_kernel", ctypes.c_int32), ("wait_timeout_us", ctypes.c_int32),
                 ("event_stats_begin", ctypes.c_void_p), ("event_stats_end", ctypes.c_void_p),
-                ("reserved", ctypes.c_int32 * 8)]
+                ("lost_copy_request", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
 
 
 _LIB = None
@@ -173,10 +173,11 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _options(stats_kernel=StatsKernel.AUTO, wait_timeout_us=0, events=None):
+def _options(stats_kernel=StatsKernel.AUTO, wait_timeout_us=0, events=None, lost_copy_request=0):
     o = _Options()
     o.stats_kernel = int(stats_kernel)
     o.wait_timeout_us = int(wait_timeout_us)
+    o.lost_copy_request = int(lost_copy_request)
     if events is not None:
         o.event_stats_begin = events[0].cuda_event
         o.event_stats_end = events[1].cuda_event
@@ -198,11 +199,13 @@ def _logit_shape(target, draft, V):
 
 def spec_verify(target, draft, tokens, lens, uniforms, temperature=1.0, greedy=False, *, V=None,
                 out=None, workspace=None, stream=None, stats_kernel=StatsKernel.AUTO,
-                wait_timeout_us=0, events=None):
+                wait_timeout_us=0, events=None, lost_copy_request=0):
     """Verify one batch on the GPU.  Returns ``(accept_len [B] int32,
     tokens [B, k_max+1] int32)`` (device tensors, valid once ``stream`` has
     run).  ``events=(begin, end)`` (torch.cuda.Event, already created)
-    brackets the row-statistics kernel."""
+    brackets the row-statistics kernel.  ``lost_copy_request`` is the
+    test-only fault injection of ``sv_options`` (1 + the request whose first
+    bulk copy is never issued; 0 = off)."""
     torch = _torch()
     B, k_max, V, dt, row_stride = _logit_shape(target, draft, V)
     dev = target.device
@@ -215,7 +218,7 @@ def spec_verify(target, draft, tokens, lens, uniforms, temperature=1.0, greedy=F
     if workspace is None:
         workspace = torch.empty(max(lib.spec_verify_workspace_bytes(ctypes.byref(shape)), 256),
                                 dtype=torch.uint8, device=dev)
-    opts = _options(stats_kernel, wait_timeout_us, events)
+    opts = _options(stats_kernel, wait_timeout_us, events, lost_copy_request)
     st = lib.spec_verify_ex(
         ctypes.byref(shape), _dev_ptr(target, what="target"), _dev_ptr(draft, what="draft"),
         _dev_ptr(tokens, torch.int32, "draft_tokens"), _dev_ptr(lens, torch.int32, "draft_lens"),

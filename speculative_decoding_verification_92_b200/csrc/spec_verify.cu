@@ -268,6 +268,8 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     sp.use_draft = (a.draft != nullptr && !greedy) ? 1 : 0;
     const int tmo = a.opts ? a.opts->wait_timeout_us : 0;
     sp.timeout_ns = tmo > 0 ? uint64_t(tmo) * 1000ull : kDefaultTimeoutNs;
+    const int lost = a.opts ? a.opts->lost_copy_request : 0;
+    sp.lost_copy_partial = lost > 0 ? int64_t(lost - 1) * (2 * s.k_max + 1) * plan.C : -1;
 
     cudaError_t e = cudaSuccess;
     if (a.opts && a.opts->event_stats_begin)
@@ -401,8 +403,9 @@ sv_status run(const Call& a) {
     if (!shape_ok(a.shape, &why)) return why;
     const sv_shape& s = *a.shape;
     if (a.opts) {
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 7; ++i)
             if (a.opts->reserved[i] != 0) return SV_EINVAL;
+        if (a.opts->lost_copy_request < 0 || a.opts->lost_copy_request > s.B) return SV_EINVAL;
         if (a.opts->stats_kernel < SV_STATS_AUTO || a.opts->stats_kernel > SV_STATS_FUSED) return SV_EINVAL;
         if (a.opts->wait_timeout_us < 0) return SV_EINVAL;
     }
@@ -438,6 +441,7 @@ sv_status run(const Call& a) {
     int variant = a.opts ? a.opts->stats_kernel : SV_STATS_AUTO;
     if (variant == SV_STATS_AUTO) variant = rows_aligned ? SV_STATS_TMA : SV_STATS_SCALAR;
     if ((variant == SV_STATS_TMA || variant == SV_STATS_VEC16) && !rows_aligned) return SV_EINVAL;
+    if (a.opts && a.opts->lost_copy_request != 0 && variant != SV_STATS_TMA) return SV_EUNSUPPORTED;
     if (variant == SV_STATS_FUSED) {
         if (!fused_ok(a, plan, rows_aligned)) return SV_EINVAL;
         return s.dtype == SV_BF16 ? run_fused<bf16_bits>(a, plan, *dev) : run_fused<float>(a, plan, *dev);

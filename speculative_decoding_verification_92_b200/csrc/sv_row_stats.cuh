@@ -65,6 +65,7 @@ struct StatsParams {
     float scale;                  // log2(e) / T
     int32_t use_draft;            // draft rows are part of the work
     uint64_t timeout_ns;          // bound on each barrier wait (TMA variant)
+    int64_t lost_copy_partial;    // test fault injection: this item's first stage is never copied; -1 = off
 };
 
 struct ItemDesc {
@@ -431,6 +432,10 @@ row_stats_tma_kernel(const StatsParams p) {
                     if (!ok) *abort_flag = 1;
                     if (*abort_flag) {
                         stop = true;
+                    } else if (sub == 0 && d.partial_idx == p.lost_copy_partial) {
+                        // injected fault: the stage is neither armed nor copied, so
+                        // the consumers' bounded wait on it runs out; last_phase[slot]
+                        // keeps the previous (completed) phase for the drain below
                     } else {
                         const int64_t off = int64_t(sub) * kStageBytes;
                         const int64_t left = tma_bytes - off;

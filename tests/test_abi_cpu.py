@@ -127,6 +127,10 @@ def test_bad_options():
     o = _Options()
     o.wait_timeout_us = -5
     assert call(opts=o) == Status.EINVAL
+    for r in (-1, 5):                      # names no request of the B = 4 batch
+        o = _Options()
+        o.lost_copy_request = r
+        assert call(opts=o) == Status.EINVAL
 
 
 def test_greedy_needs_no_uniforms_or_temperature_and_empty_batch_is_ok():
