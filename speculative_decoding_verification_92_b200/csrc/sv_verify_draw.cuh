@@ -1,7 +1,8 @@
 // sv_verify_draw.cuh -- K2, acceptance scan and the final draw.
 //
-// One thread-block cluster of C CTAs per request; CTA c of the cluster owns
-// vocabulary chunk c of the row that the final draw uses.
+// One thread-block cluster per request, of C2 = ceil(C / R) CTAs; CTA c of
+// the cluster owns the R consecutive vocabulary chunks c*R .. c*R+R-1 of the
+// row that the final draw uses.
 //
 //  1. validate draft_lens[b] and the first L drafted ids (bad values never
 //     cause an access: the request is reported with out_accept_len = -1);
@@ -15,25 +16,24 @@
 //  4. final draw on row j with uniforms[b][k_max]:
 //       bonus (j == L):     w = p_L, chunk sums straight from the K1 partials;
 //       one-hot rejection:  w = p_j with the drafted id removed, same;
-//       draft rejection:    w = max(0, p_j - q_j); every CTA computes its
-//                           chunk's sum, the sums are exchanged through
-//                           distributed shared memory and a cluster barrier;
-//     every CTA locates the chunk holding u*W.  In that CTA the chunk is read
-//     once with coalesced 16-byte loads (warp w owns a contiguous run of
-//     vectors, lane l the vectors w*WV + 32*it + l); each lane keeps the
-//     weight sum of each of its vectors in registers, so the crossing is
-//     found by narrowing down warp -> iteration -> lane (block scan of warp
-//     totals, a running sum over iterations, a warp scan over lanes), and only
-//     the one vector holding C_t > u*W is read again to pick the element.  In
-//     the residual case the same pass also yields the chunk sum that is
-//     exchanged, so the chosen CTA does not read its chunk twice.  Rows that
-//     do not start on a 16-byte boundary (or very long chunks) use a slower
-//     pass over contiguous per-thread segments instead.
+//       draft rejection:    w = max(0, p_j - q_j); every CTA runs the draw
+//                           pass over its chunks and the chunk sums are
+//                           exchanged through distributed shared memory and
+//                           a cluster barrier;
+//     every CTA locates the chunk k* holding u*W, and only its owner goes on.
+//  5. inverse CDF inside chunk k*.  The draw pass streams a chunk through a
+//     small shared-memory ring filled by 16-byte cp.async copies (each thread
+//     reads back only what it copied, so the ring needs no block barrier) and
+//     keeps one weight sum per segment of 32 vectors.  A warp then picks the
+//     segment (scan over lanes), re-reads that one segment (one vector per
+//     lane) to pick the vector, and the element from the lane's registers.
+//     For a draft rejection the pass of step 4 already holds chunk k*'s
+//     segment sums; a bonus or one-hot draw runs the pass over chunk k*
+//     alone.  Rows that do not start on a 16-byte boundary (or very long
+//     chunks) use contiguous per-thread segments, a block scan and one walk.
 //
-// Shared memory stays small (the row partials and per-draft scalars), so
-// many clusters are resident at once.  A request's cluster has ceil(C / R)
-// CTAs, each owning R consecutive chunks, with R chosen so that the whole
-// batch fits in about one wave.  The kernel is a programmatic dependent of the
+// R is the fewest chunks per CTA that fit the batch in about two waves of the
+// resident CTAs.  The kernel is a programmatic dependent of the
 // row-statistics kernel (which signals at the end of each CTA): its
 // input-only prologue overlaps that kernel's last CTAs, and it waits for the
 // kernel's completion (griddepcontrol.wait) before reading the partials.
