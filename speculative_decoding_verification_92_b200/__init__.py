@@ -23,11 +23,13 @@ from pathlib import Path
 __all__ = [
     "Status", "StatsKernel", "SpecVerifyError", "library", "workspace_bytes",
     "spec_verify", "spec_verify_stats", "spec_verify_accept_sim", "spec_verify_host", "host_staging_bytes",
-    "abi_version", "F32", "BF16",
+    "abi_version", "F32", "BF16", "MAX_K", "MAX_V",
 ]
 
 F32 = 0
 BF16 = 1
+MAX_K = 1024      # SV_MAX_K of the C header: largest supported k_max
+MAX_V = 393216    # SV_MAX_V of the C header: largest supported vocabulary
 
 
 class Status(enum.IntEnum):

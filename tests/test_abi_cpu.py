@@ -98,8 +98,8 @@ def call(shape=None, target=FAKE, draft=None, tokens=FAKE, lens=None, uniforms=F
     (dict(shape=_Shape(4, -2, 10, sv.F32, 0)), Status.EINVAL),
     (dict(shape=_Shape(4, 4, 10, sv.F32, 9)), Status.EINVAL),
     (dict(shape=_Shape(4, 4, 10, 5, 0)), Status.EUNSUPPORTED),
-    (dict(shape=_Shape(4, 1025, 10, sv.F32, 0)), Status.EUNSUPPORTED),
-    (dict(shape=_Shape(4, 4, 393217, sv.F32, 0)), Status.EUNSUPPORTED),
+    (dict(shape=_Shape(4, sv.MAX_K + 1, 10, sv.F32, 0)), Status.EUNSUPPORTED),
+    (dict(shape=_Shape(4, 4, sv.MAX_V + 1, sv.F32, 0)), Status.EUNSUPPORTED),
     (dict(target=None), Status.EINVAL),
     (dict(tokens=None), Status.EINVAL),
     (dict(out_len=None), Status.EINVAL),
@@ -164,3 +164,13 @@ def test_python_binding_rejects_host_tensors():
     t = torch.zeros(2, 3, 10)
     with pytest.raises(ValueError):
         sv.spec_verify(t, None, torch.zeros(2, 2, dtype=torch.int32), None, torch.zeros(2, 3))
+
+
+def test_size_limits_match_the_header():
+    text = (Path(__file__).resolve().parents[1] / "include" / "spec_verify.h").read_text()
+    assert int(re.search(r"#define SV_MAX_K (\d+)", text).group(1)) == sv.MAX_K
+    assert int(re.search(r"#define SV_MAX_V (\d+)", text).group(1)) == sv.MAX_V
+    lib = sv.library()
+    for dt in (sv.F32, sv.BF16):
+        assert lib.spec_verify_workspace_bytes(ctypes.byref(_Shape(3, sv.MAX_K, sv.MAX_V, dt, 0))) > 0
+        assert lib.spec_verify_workspace_bytes(ctypes.byref(_Shape(3, 2, sv.MAX_V + 1, dt, 0))) == 0

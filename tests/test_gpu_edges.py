@@ -2,7 +2,8 @@
 vocabulary tails, tiny and single-token vocabularies, empty drafts, padded
 and misaligned rows, temperatures, greedy ties across chunk boundaries,
 extreme uniforms, invalid ids / lengths, large batches split over several
-launches, and closed forms of the rule."""
+launches, the largest vocabulary and draft length, and closed forms of the
+rule."""
 import numpy as np
 import pytest
 import torch
@@ -144,6 +145,33 @@ def test_invalid_requests_are_reported_not_read():
     compare(w, g_len, g_tok, o, diag=o)
     assert list(g_len[[0, 1, 3, 4]]) == [-1, -1, -1, -1]
     assert g_len[2] >= 0 and g_len[5] >= 0
+
+
+@pytest.mark.parametrize("dtype", [F32, BF16])
+def test_largest_vocabulary(dtype):
+    # V = MAX_V: 8 chunks of 192 KiB (fp32, beyond the ring draw: the segment
+    # draw with 16-byte loads) or of 96 KiB (bf16, the ring draw)
+    # heavy-tailed logits (sigma 4): the mass sits on a few hundred ids spread
+    # over the whole row, so most draws are far from a near-tie and compare
+    # exactly, while the chunk and segment sums still span every chunk
+    w = make_workload(B=6, k_max=2, V=sv.MAX_V, dtype=dtype, seed=61, z_sigma=4.0, boost=0.0,
+                      draft_noise=0.5, lens=[2, 1, 0, 2, 2, 1])
+    o = check(w)
+    assert np.count_nonzero(o["flags"] & 3) <= 2
+    check(w, greedy=True)
+
+
+def test_largest_draft_length():
+    # k_max = MAX_K: four drafts per draw-kernel thread; one request accepts
+    # all 1024 drafts (identical draft, bonus from row 1024), the others stop
+    # early or at their own length
+    w = make_workload(B=3, k_max=sv.MAX_K, V=256, dtype=F32, seed=62, boost=3.0, draft_noise=0.3,
+                      lens=[sv.MAX_K, 1000, 517])
+    w.draft[0] = w.target[0, :sv.MAX_K]
+    check(w)
+    check(w, greedy=True)
+    g_len, _ = run_gpu(w)
+    assert g_len[0] == sv.MAX_K
 
 
 def test_many_requests_span_several_launches():
