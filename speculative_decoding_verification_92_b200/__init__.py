@@ -168,6 +168,20 @@ def _dev_ptr(t, dtype=None, what="tensor"):
     return t.data_ptr()
 
 
+def _check_shapes(device, **named):
+    """Every given tensor must have exactly its expected shape (the library
+    reads that many elements through the raw pointer) and, when ``device`` is
+    given, live on that device.  ``named`` maps a name to (tensor, shape);
+    None tensors are skipped, a None shape checks the device only."""
+    for what, (t, shape) in named.items():
+        if t is None:
+            continue
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{what} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+        if device is not None and t.device != device:
+            raise ValueError(f"{what} is on {t.device}, the logits on {device}")
+
+
 def _stream_handle(stream):
     torch = _torch()
     if stream is None:
@@ -215,6 +229,10 @@ def spec_verify(target, draft, tokens, lens, uniforms, temperature=1.0, greedy=F
         out = (torch.empty(B, dtype=torch.int32, device=dev),
                torch.empty(B, k_max + 1, dtype=torch.int32, device=dev))
     out_len, out_tok = out
+    _check_shapes(dev, draft_tokens=(tokens, (B, k_max)), draft_lens=(lens, (B,)),
+                  uniforms=(None if greedy else uniforms, (B, k_max + 1)),
+                  out_accept_len=(out_len, (B,)), out_tokens=(out_tok, (B, k_max + 1)),
+                  draft=(draft, None), workspace=(workspace, None))
     shape = _shape(B, k_max, V, dt, row_stride)
     lib = library()
     if workspace is None:
@@ -244,6 +262,7 @@ def spec_verify_stats(target, draft, tokens, lens, temperature=1.0, *, V=None, w
     lse_d = torch.empty(B, k_max, dtype=torch.float32, device=dev)
     p = torch.empty(B, k_max, dtype=torch.float32, device=dev)
     q = torch.empty(B, k_max, dtype=torch.float32, device=dev)
+    _check_shapes(dev, draft_tokens=(tokens, (B, k_max)), draft_lens=(lens, (B,)))
     shape = _shape(B, k_max, V, dt, row_stride)
     lib = library()
     if workspace is None:
@@ -275,6 +294,8 @@ def spec_verify_accept_sim(target, draft, tokens, lens, uniforms=None, temperatu
     e = torch.empty(B, dtype=torch.float32, device=dev)
     j = torch.empty(B, dtype=torch.int32, device=dev) if uniforms is not None else None
     w = torch.empty(B, k_max, dtype=torch.float32, device=dev) if uniforms is not None else None
+    _check_shapes(dev, draft_tokens=(tokens, (B, k_max)), draft_lens=(lens, (B,)),
+                  uniforms=(uniforms, (B, k_max + 1)))
     shape = _shape(B, k_max, V, dt, row_stride)
     lib = library()
     if workspace is None:
@@ -317,6 +338,9 @@ def spec_verify_host(target, draft, tokens, lens, uniforms, temperature=1.0, gre
     if out is None:
         out = (torch.empty(B, dtype=torch.int32, pin_memory=True),
                torch.empty(B, k_max + 1, dtype=torch.int32, pin_memory=True))
+    _check_shapes(None, draft_tokens=(tokens, (B, k_max)), draft_lens=(lens, (B,)),
+                  uniforms=(None if greedy else uniforms, (B, k_max + 1)),
+                  out_accept_len=(out[0], (B,)), out_tokens=(out[1], (B, k_max + 1)))
     if staging is None:
         n = lib.spec_verify_host_staging_bytes(ctypes.byref(shape), int(draft is not None), int(lens is not None))
         staging = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)

@@ -166,6 +166,26 @@ def test_python_binding_rejects_host_tensors():
         sv.spec_verify(t, None, torch.zeros(2, 2, dtype=torch.int32), None, torch.zeros(2, 3))
 
 
+@pytest.mark.parametrize("bad,msg", [
+    (dict(tokens=(3, 3)), "draft_tokens must have shape"),
+    (dict(lens=(4,)), "draft_lens must have shape"),
+    (dict(uniforms=(3, 4)), "uniforms must have shape"),
+    (dict(out_tok=(3, 4)), "out_tokens must have shape"),
+    (dict(out_len=(2,)), "out_accept_len must have shape"),
+])
+def test_python_binding_checks_shapes_before_any_call(bad, msg):
+    # the library reads exactly B*k ids, B lengths and B*(k+1) uniforms
+    # through raw pointers, so a wrongly shaped tensor must never reach it
+    import torch
+    B, k, V = 3, 4, 64
+    shapes = dict(tokens=(B, k), lens=(B,), uniforms=(B, k + 1), out_len=(B,), out_tok=(B, k + 1))
+    shapes.update(bad)
+    i32 = lambda key: torch.zeros(shapes[key], dtype=torch.int32)
+    with pytest.raises(ValueError, match=msg):
+        sv.spec_verify(torch.zeros(B, k + 1, V), torch.zeros(B, k, V), i32("tokens"), i32("lens"),
+                       torch.zeros(shapes["uniforms"]), out=(i32("out_len"), i32("out_tok")))
+
+
 def test_size_limits_match_the_header():
     text = (Path(__file__).resolve().parents[1] / "include" / "spec_verify.h").read_text()
     assert int(re.search(r"#define SV_MAX_K (\d+)", text).group(1)) == sv.MAX_K
