@@ -28,6 +28,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import itertools
 import json
 import math
 import os
@@ -360,11 +361,29 @@ def run_host(args):
     for p, c in items[:2000]:
         d = ng.draft(p, c, 16)
         accepted.append(len(d))
+
+    # batched drafting of whole verification batches (B = 128 requests per
+    # call, the n-gram workload's batch) straight into draft_tokens / draft_lens
+    Bq = 128
+    batches = [([p for p, _ in items[i:i + Bq]], [c for _, c in items[i:i + Bq]])
+               for i in range(0, len(items) - Bq + 1, Bq)]
+
+    def batch_rate(threads):
+        n, t0 = 0, time.perf_counter()
+        for pids, cs in itertools.cycle(batches):
+            ng.draft_batch(pids, cs, 16, n_threads=threads)
+            n += Bq
+            if time.perf_counter() - t0 > 3.0:
+                break
+        return n / (time.perf_counter() - t0)
+    batch_1, batch_all = batch_rate(1), batch_rate(0)
     line = {
         "metric": "host n-gram draft lookups/s (k=16), 1 core", "value": ng_rate, "unit": "lookups/s",
         "data": "synthetic", "config": {"workload": f"{P} prompts x {R} rollouts x {T} tokens, W={W} steps, "
                                                     "10% token changes per rollout", "max_n": 6, "k": 16},
         "ngram_candidates_per_s": ng_cand, "suffix_draft_per_s": sx_rate, "prefetch_allocations_per_s": pf_rate,
+        "ngram_batch_drafts_per_s": {"batch": Bq, "threads_1": batch_1, "threads_all": batch_all,
+                                     "hardware_threads": os.cpu_count()},
         "table_build_s": build_s, "retained_tokens": ng.tokens, "mean_draft_len": float(np.mean(accepted)),
         "cpu_baseline": {"value": o_rate, "unit": "lookups/s", "cores": 1, "kind": "oracle",
                          "sample": f"{o_n} n-gram draft lookups with the plain-Python oracle"},

@@ -129,6 +129,38 @@ SV_API int32_t sv_suffix_candidates(const sv_suffix *t, int64_t problem_id, cons
                                     int64_t n, int32_t f, int32_t *out);
 
 /* ------------------------------------------------------------------------
+ * Batched drafting straight into the verification inputs.
+ *
+ * One call drafts for a whole batch and writes the drafted-id and length
+ * arrays of spec_verify's one-hot path (no draft logits).  Request b
+ * continues ctx[ctx_off[b] .. ctx_off[b+1]) of prompt (problem) ids[b] and
+ * drafts up to cap_b = min(k_max, max_lens[b]) tokens (k_max alone when
+ * max_lens is NULL; a cap from the draft-length controller or the request
+ * budgets goes there).  The result is exactly what the single-request draft
+ * call returns with k = cap_b:
+ *   out_tokens[b][0 .. m_b)      the drafted ids;
+ *   out_tokens[b][m_b .. k_max)  -1;
+ *   out_lens[b] = m_b.
+ * A request with no match gets m_b = 0, which spec_verify treats as no
+ * speculation (one token drawn from target row 0).
+ *
+ * Layouts: ids[B]; ctx_off[B+1], non-decreasing from ctx_off[0] >= 0, with
+ * ctx holding at least ctx_off[B] tokens; max_lens[B] or NULL; out_tokens
+ * [B][k_max] row-major; out_lens[B].  All host memory, owned by the caller.
+ * The table is only read, so requests run concurrently on up to n_threads
+ * host threads (0 = one per hardware thread; small batches use fewer).  The
+ * table must not be modified during the call.  Returns 0, or -1 on bad
+ * arguments (NULL pointers, B < 0, k_max outside [0, SV_MAX_K], decreasing
+ * offsets, a negative cap, n_threads < 0); nothing is written then.
+ */
+SV_API int32_t sv_ngram_draft_batch(const sv_ngram *t, int32_t B, const int64_t *ids, const int32_t *ctx,
+                                    const int64_t *ctx_off, int32_t k_max, const int32_t *max_lens,
+                                    int32_t n_threads, int32_t *out_tokens, int32_t *out_lens);
+SV_API int32_t sv_suffix_draft_batch(const sv_suffix *t, int32_t B, const int64_t *ids, const int32_t *ctx,
+                                     const int64_t *ctx_off, int32_t k_max, const int32_t *max_lens,
+                                     int32_t n_threads, int32_t *out_tokens, int32_t *out_lens);
+
+/* ------------------------------------------------------------------------
  * Fan-out prefetch budget [NG-FETCH].
  *
  * Observations are verification outcomes: j in [0, k] accepted drafts and the

@@ -28,6 +28,8 @@ _HOST_SIGNATURES = {
     "sv_suffix_append": (_I32, [_VP, _I64, _I64, _VP, _I64]),
     "sv_suffix_draft": (_I32, [_VP, _I64, _VP, _I64, _I32, _VP]),
     "sv_suffix_candidates": (_I32, [_VP, _I64, _VP, _I64, _I32, _VP]),
+    "sv_ngram_draft_batch": (_I32, [_VP, _I32, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _VP]),
+    "sv_suffix_draft_batch": (_I32, [_VP, _I32, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _VP]),
     "sv_prefetch_create": (_VP, [_I32, _I32, _I32]),
     "sv_prefetch_destroy": (None, [_VP]),
     "sv_prefetch_observe": (_I32, [_VP, _I32, _I32]),
@@ -60,6 +62,36 @@ def _L():
 
 def _tok(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a, dtype=np.int32).reshape(-1))
+
+
+def _draft_batch(fn, h, ids, contexts, k_max, max_lens, n_threads):
+    """Shared marshalling of the batched drafting calls: returns the
+    drafted-id array [B, k_max] (-1 padded) and the lengths [B], both int32,
+    in the layout spec_verify takes as draft_tokens / draft_lens."""
+    ids = np.ascontiguousarray(np.asarray(ids, dtype=np.int64).reshape(-1))
+    B = ids.size
+    if len(contexts) != B:
+        raise ValueError(f"{B} ids but {len(contexts)} contexts")
+    off = np.zeros(B + 1, np.int64)
+    np.cumsum(np.fromiter((len(c) for c in contexts), np.int64, count=B), out=off[1:])
+    # one concatenation (and one conversion to int32) for the whole batch
+    parts = [c for c in contexts if len(c)]          # an empty list would come in as float64
+    flat = np.concatenate(parts, dtype=np.int32, casting="same_kind") if parts else np.zeros(1, np.int32)
+    if flat.size != off[-1]:
+        raise ValueError("every context must be a flat sequence of token ids")
+    caps = None
+    if max_lens is not None:
+        caps = np.ascontiguousarray(np.asarray(max_lens, dtype=np.int32).reshape(-1))
+        if caps.size != B:
+            raise ValueError(f"{B} ids but {caps.size} max_lens")
+    tokens = np.empty((B, int(k_max)), np.int32)
+    lens = np.empty(B, np.int32)
+    rc = fn(h, B, ids.ctypes.data, flat.ctypes.data, off.ctypes.data, int(k_max),
+            None if caps is None else caps.ctypes.data, int(n_threads),
+            tokens.ctypes.data if tokens.size else None, lens.ctypes.data)
+    if rc != 0:
+        raise ValueError("batched drafting rejected its arguments")
+    return tokens, lens
 
 
 class _Handle:
@@ -106,6 +138,13 @@ class NgramDrafter(_Handle):
             raise ValueError("sv_ngram_draft rejected its arguments")
         return out[:n].copy()
 
+    def draft_batch(self, prompt_ids, contexts, k_max: int, max_lens=None, n_threads: int = 0):
+        """Drafts for a whole batch in one call: ``(draft_tokens [B, k_max],
+        draft_lens [B])`` int32, -1 padded, ready for spec_verify without
+        draft logits.  ``max_lens`` caps each request (controller length or
+        budget); ``n_threads`` 0 uses the hardware threads."""
+        return _draft_batch(_L().sv_ngram_draft_batch, self._h, prompt_ids, contexts, k_max, max_lens, n_threads)
+
     def candidates(self, prompt_id: int, context, f: int) -> np.ndarray:
         c = _tok(context)
         out = np.empty(max(int(f), 1), np.int32)
@@ -145,6 +184,10 @@ class SuffixDrafter(_Handle):
         if n < 0:
             raise ValueError("sv_suffix_draft rejected its arguments")
         return out[:n].copy()
+
+    def draft_batch(self, problem_ids, contexts, k_max: int, max_lens=None, n_threads: int = 0):
+        """Batched drafting, as NgramDrafter.draft_batch."""
+        return _draft_batch(_L().sv_suffix_draft_batch, self._h, problem_ids, contexts, k_max, max_lens, n_threads)
 
     def candidates(self, problem_id: int, context, f: int) -> np.ndarray:
         c = _tok(context)

@@ -337,3 +337,71 @@ def test_ngram_speculation_on_repeating_rollouts():
 
     rates = [accepted_per_cycle(p) for p in (0.5, 0.81, 1.0)]
     assert rates[0] < rates[1] < rates[2] and rates[2] == 16.0
+
+
+# ---------------------------------------------------------------------------
+# batched drafting into spec_verify's drafted-id / length arrays
+
+@pytest.mark.parametrize("which", ["ngram", "suffix"])
+def test_batched_drafting_matches_the_oracle_for_every_thread_count(which):
+    rng = np.random.default_rng(400)
+    if which == "ngram":
+        o, c = ho.NgramOracle(5, 3), host.NgramDrafter(5, 3)
+        for step in range(3):
+            o.begin_step()
+            c.begin_step()
+            for pid in range(6):
+                toks = markov_stream(rng, int(rng.integers(20, 80)), 14)
+                o.add(pid, toks)
+                c.add(pid, toks)
+    else:
+        o, c = ho.SuffixOracle(6), host.SuffixDrafter(6)
+        for pid in range(6):
+            for sid in range(3):
+                toks = markov_stream(rng, int(rng.integers(20, 80)), 14)
+                o.append(pid, sid, toks)
+                c.append(pid, sid, toks)
+    B, k_max = 200, 12
+    ids = rng.integers(0, 8, size=B)                  # prompts 6 and 7 have no history
+    ctxs = [markov_stream(rng, int(rng.integers(0, 15)), 14) for _ in range(B)]
+    ctxs[3], ctxs[5] = [], np.zeros(0, np.int64)       # empty contexts draft nothing
+    caps = rng.integers(0, 20, size=B)                # some above k_max, some 0
+    results = [c.draft_batch(ids, ctxs, k_max, caps, n_threads=nt) for nt in (1, 3, 0)]
+    for tok, lens in results[1:]:
+        assert np.array_equal(tok, results[0][0]) and np.array_equal(lens, results[0][1])
+    tok, lens = results[0]
+    assert tok.shape == (B, k_max) and tok.dtype == np.int32 and lens.dtype == np.int32
+    for b in range(B):
+        want = o.draft(int(ids[b]), ctxs[b], int(min(k_max, caps[b])))
+        assert list(tok[b, :lens[b]]) == want and np.all(tok[b, lens[b]:] == -1)
+    assert (lens == 0).any() and (lens == k_max).any()
+    # without caps every request may use k_max
+    tok2, lens2 = c.draft_batch(ids, ctxs, k_max)
+    assert np.all(lens2 >= lens)
+
+
+def test_batched_drafting_rejects_bad_arguments():
+    import ctypes
+    d = host.NgramDrafter(3, 2)
+    d.begin_step()
+    d.add(0, [1, 2, 3, 4])
+    lib = host._L()
+    ids = np.zeros(2, np.int64)
+    ctx = np.array([1, 2, 3], np.int32)
+    tok = np.zeros((2, 4), np.int32)
+    lens = np.zeros(2, np.int32)
+    P = lambda a: a.ctypes.data
+
+    def call(off=(0, 1, 3), k=4, caps=None, nt=1, B=2, handle=d._h):
+        off = np.asarray(off, np.int64)
+        return lib.sv_ngram_draft_batch(handle, B, P(ids), P(ctx), P(off), k,
+                                        None if caps is None else P(np.asarray(caps, np.int32)), nt, P(tok), P(lens))
+    assert call() == 0 and list(lens) == [3, 1]      # [1] -> 2 3 4; [2 3] -> 4
+    tok[:] = 7
+    for bad in (dict(off=(0, 2, 1)), dict(off=(-1, 1, 3)), dict(k=-1), dict(k=1025), dict(caps=(1, -1)),
+                dict(nt=-2), dict(B=-1), dict(handle=None)):
+        assert call(**bad) == -1
+    assert np.all(tok == 7)                           # nothing written on rejection
+    assert call(B=0) == 0
+    with pytest.raises(ValueError):
+        d.draft_batch([0, 0], [[1]], 4)               # one context for two ids
