@@ -33,7 +33,8 @@ def test_lost_copy_times_out_and_the_context_stays_usable(V, dtype, victim, gree
     clean = verify(d, w, greedy)
     assert np.all(clean[0] >= 0)
 
-    n, t = verify(d, w, greedy, wait_timeout_us=2000, lost_copy_request=victim + 1)
+    # 20 ms: long against any normal wait (microseconds), short for a test
+    n, t = verify(d, w, greedy, wait_timeout_us=20000, lost_copy_request=victim + 1)
     assert n[victim] == -2 and np.all(t[victim] == -1)
     # other requests: unaffected, or lost with the rest of that CTA's later work
     lost = n == -2
