@@ -377,6 +377,33 @@ def run_host(args):
                 break
         return n / (time.perf_counter() - t0)
     batch_1, batch_all = batch_rate(1), batch_rate(0)
+
+    # fan-out prefetch: the whole pipeline (budget, drafting ahead, serving
+    # with a synchronous fallback) along fresh rollouts of the same prompts,
+    # verified by prefix match against them
+    fp = host.FanoutPrefetcher(ng, k=16, budget=16, fmax=16, window=256)
+    preds, t_prep, n_steps = [], 0.0, 0
+    for p in range(8):
+        text = base[p].copy()
+        m = rng.random(T) < 0.1
+        text[m] = rng.integers(0, V, int(m.sum()))
+        text = [int(x) for x in text]
+        pos = 8
+        while pos < T - 18:
+            ctx = text[:pos]
+            d = [int(x) for x in ng.draft(p, ctx, 16)]
+            t0 = time.perf_counter()
+            preds.append(fp.prepare(n_steps, p, ctx, d))
+            t_prep += time.perf_counter() - t0
+            j = 0
+            while j < len(d) and d[j] == text[pos + j]:
+                j += 1
+            fp.next_draft(n_steps, j, text[pos + j])
+            n_steps += 1
+            pos += j + 1
+    fanout = {"steps": n_steps, "hit_rate": fp.hits / max(n_steps, 1),
+              "predicted_hit_rate": float(np.mean(preds)) if preds else 0.0,
+              "prepare_us": 1e6 * t_prep / max(n_steps, 1)}
     line = {
         "metric": "host n-gram draft lookups/s (k=16), 1 core", "value": ng_rate, "unit": "lookups/s",
         "data": "synthetic", "config": {"workload": f"{P} prompts x {R} rollouts x {T} tokens, W={W} steps, "
@@ -384,6 +411,7 @@ def run_host(args):
         "ngram_candidates_per_s": ng_cand, "suffix_draft_per_s": sx_rate, "prefetch_allocations_per_s": pf_rate,
         "ngram_batch_drafts_per_s": {"batch": Bq, "threads_1": batch_1, "threads_all": batch_all,
                                      "hardware_threads": os.cpu_count()},
+        "fanout_prefetch": fanout,
         "table_build_s": build_s, "retained_tokens": ng.tokens, "mean_draft_len": float(np.mean(accepted)),
         "cpu_baseline": {"value": o_rate, "unit": "lookups/s", "cores": 1, "kind": "oracle",
                          "sample": f"{o_n} n-gram draft lookups with the plain-Python oracle"},

@@ -191,6 +191,36 @@ SV_API int32_t sv_prefetch_estimates(const sv_prefetch *p, double *P_j, double *
 SV_API double sv_prefetch_allocate(const sv_prefetch *p, int32_t budget, int32_t *out_f);
 
 /* ------------------------------------------------------------------------
+ * Fan-out prefetch of the next draft [NG-FETCH].
+ *
+ * While the GPU verifies draft d[0..L) of a request that continues
+ * context[0..n), the host drafts ahead for the outcomes the budget covers.
+ * After outcome (j, b) -- j drafts accepted, b the emitted token -- the
+ * request continues context + d[0..j) + b.  Branch j takes the f[j]
+ * top-ranked candidates b for the token after context + d[0..j) (the
+ * sv_ngram_candidates ranking, the same ranking whose rank of the actual b
+ * feeds sv_prefetch_observe), and each (j, b) gets the next draft
+ * sv_ngram_draft(context + d[0..j) + b, k).  Entries are written in order of
+ * j, then candidate rank:
+ *   out_j[e], out_b[e], out_tokens[e][0..k) (-1 padded), out_lens[e];
+ * at most max_entries of them.  f[0..L] (from sv_prefetch_allocate with this
+ * request's L as k) may ask for more candidates than a branch has; such a
+ * branch gets what exists.  Returns the entry count, or -1 on bad arguments
+ * (NULL pointers, n < 0, L < 0, L > SV_MAX_K, a negative f[j], k outside
+ * [0, SV_MAX_K], max_entries < 0).  All arrays are host memory owned by the
+ * caller; the table is only read.
+ *
+ * When verification reports (j, b), sv_prefetch_find returns the entry that
+ * holds its next draft (a hit) or -1 (a miss: draft synchronously).
+ */
+SV_API int32_t sv_ngram_prefetch(const sv_ngram *t, int64_t prompt_id, const int32_t *context, int64_t n,
+                                 const int32_t *draft, int32_t L, const int32_t *f, int32_t k,
+                                 int32_t max_entries, int32_t *out_j, int32_t *out_b, int32_t *out_tokens,
+                                 int32_t *out_lens);
+/* The entry e < count with out_j[e] == j and out_b[e] == b, or -1. */
+SV_API int32_t sv_prefetch_find(const int32_t *out_j, const int32_t *out_b, int32_t count, int32_t j, int32_t b);
+
+/* ------------------------------------------------------------------------
  * Adaptive draft length [ER-LEN].
  *
  * Candidate lengths ascending (e.g. 5, 7, 9, 11); the controller starts at

@@ -180,6 +180,20 @@ def expected_coverage(P, cov, f):
     return sum(P[j] * cov[j][f[j]] for j in range(len(f)))
 
 
+def prefetch_drafts(drafter, pid, ctx, draft, f, k):
+    """Fan-out prefetch ("🚰 真正的瓶颈不在算法，在流水线"): for each branch j (j drafts
+    accepted) and each of its f[j] best-ranked candidates b for the next
+    token, the draft that would follow context + draft[:j] + [b], computed
+    before the outcome is known.  Returns {(j, b): draft}."""
+    ctx, draft = [int(x) for x in ctx], [int(x) for x in draft]
+    out = {}
+    for j in range(len(draft) + 1):
+        branch = ctx + draft[:j]
+        for b in drafter.candidates(pid, branch, f[j]):
+            out[(j, int(b))] = [int(x) for x in drafter.draft(pid, branch + [int(b)], k)]
+    return out
+
+
 # --------------------------------------------------------------------------
 # draft length, block efficiency, switch, budgets
 

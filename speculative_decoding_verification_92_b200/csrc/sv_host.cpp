@@ -524,6 +524,58 @@ double sv_prefetch_allocate(const sv_prefetch* p, int32_t budget, int32_t* out_f
     return total;
 }
 
+// ---------------------------------------------------------------------------
+// Fan-out prefetch of the next draft: for every covered outcome (j, b), the
+// draft that follows context + d[0..j) + b, computed ahead of the outcome.
+
+int32_t sv_ngram_prefetch(const sv_ngram* t, int64_t prompt_id, const int32_t* context, int64_t n,
+                          const int32_t* draft, int32_t L, const int32_t* f, int32_t k, int32_t max_entries,
+                          int32_t* out_j, int32_t* out_b, int32_t* out_tokens, int32_t* out_lens) {
+    if (!t || n < 0 || (n > 0 && !context) || L < 0 || L > SV_MAX_K || (L > 0 && !draft) || !f || k < 0 ||
+        k > SV_MAX_K || max_entries < 0)
+        return -1;
+    for (int32_t j = 0; j <= L; ++j)
+        if (f[j] < 0) return -1;
+    if (max_entries > 0 && (!out_j || !out_b || !out_lens || (k > 0 && !out_tokens))) return -1;
+    try {
+        std::vector<int32_t> ctx;  // context + d[0..j), then + b while drafting
+        ctx.reserve(static_cast<size_t>(n) + L + 1);
+        ctx.assign(context, context + n);
+        std::vector<int32_t> cand;
+        int32_t e = 0;
+        for (int32_t j = 0; j <= L && e < max_entries; ++j) {
+            if (j > 0) ctx.push_back(draft[j - 1]);
+            const int32_t want = std::min(f[j], max_entries - e);
+            if (want == 0) continue;
+            cand.resize(static_cast<size_t>(want));
+            const int32_t nc = sv_ngram_candidates(t, prompt_id, ctx.data(), static_cast<int64_t>(ctx.size()), want,
+                                                   cand.data());
+            for (int32_t r = 0; r < nc; ++r, ++e) {
+                ctx.push_back(cand[r]);
+                int32_t* row = k > 0 ? out_tokens + static_cast<int64_t>(e) * k : nullptr;
+                int32_t m = k > 0 ? sv_ngram_draft(t, prompt_id, ctx.data(), static_cast<int64_t>(ctx.size()), k, row)
+                                  : 0;
+                m = std::max(m, 0);
+                for (int32_t i = m; i < k; ++i) row[i] = -1;
+                ctx.pop_back();
+                out_j[e] = j;
+                out_b[e] = cand[r];
+                out_lens[e] = m;
+            }
+        }
+        return e;
+    } catch (...) {  // allocation failure: nothing may cross the C boundary
+        return -1;
+    }
+}
+
+int32_t sv_prefetch_find(const int32_t* out_j, const int32_t* out_b, int32_t count, int32_t j, int32_t b) {
+    if (!out_j || !out_b) return -1;
+    for (int32_t e = 0; e < count; ++e)
+        if (out_j[e] == j && out_b[e] == b) return e;
+    return -1;
+}
+
 // ===========================================================================
 // Draft-length controller, block efficiency, speculation switch.
 

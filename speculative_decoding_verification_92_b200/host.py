@@ -35,6 +35,8 @@ _HOST_SIGNATURES = {
     "sv_prefetch_observe": (_I32, [_VP, _I32, _I32]),
     "sv_prefetch_estimates": (_I32, [_VP, _VP, _VP]),
     "sv_prefetch_allocate": (_F64, [_VP, _I32, _VP]),
+    "sv_ngram_prefetch": (_I32, [_VP, _I64, _VP, _I64, _VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP]),
+    "sv_prefetch_find": (_I32, [_VP, _VP, _I32, _I32, _I32]),
     "sv_draft_len_create": (_VP, [_VP, _I32, _F64, _F64, _I32]),
     "sv_draft_len_destroy": (None, [_VP]),
     "sv_draft_len_current": (_I32, [_VP]),
@@ -138,6 +140,24 @@ class NgramDrafter(_Handle):
             raise ValueError("sv_ngram_draft rejected its arguments")
         return out[:n].copy()
 
+    def prefetch(self, prompt_id: int, context, draft, f, k: int = 16, max_entries=None) -> dict:
+        """Next drafts for the verification outcomes that the allocation
+        ``f`` (one entry per branch j = 0..len(draft)) covers, drafted before
+        the outcome is known: ``{(j, b): ids}`` (sv_ngram_prefetch)."""
+        c, d = _tok(context), _tok(draft)
+        fa = np.ascontiguousarray(np.asarray(f, dtype=np.int32).reshape(-1))
+        if fa.size != d.size + 1:
+            raise ValueError(f"f needs {d.size + 1} entries (branches j = 0..{d.size}), got {fa.size}")
+        cap = int(fa.clip(min=0).sum()) if max_entries is None else int(max_entries)
+        oj, ob, ol = (np.empty(max(cap, 1), np.int32) for _ in range(3))
+        ot = np.empty((max(cap, 1), max(int(k), 1)), np.int32)
+        n = _L().sv_ngram_prefetch(self._h, int(prompt_id), c.ctypes.data, c.size, d.ctypes.data, d.size,
+                                   fa.ctypes.data, int(k), cap, oj.ctypes.data, ob.ctypes.data, ot.ctypes.data,
+                                   ol.ctypes.data)
+        if n < 0:
+            raise ValueError("sv_ngram_prefetch rejected its arguments")
+        return {(int(oj[e]), int(ob[e])): ot[e, :ol[e]].copy() for e in range(n)}
+
     def draft_batch(self, prompt_ids, contexts, k_max: int, max_lens=None, n_threads: int = 0):
         """Drafts for a whole batch in one call: ``(draft_tokens [B, k_max],
         draft_lens [B])`` int32, -1 padded, ready for spec_verify without
@@ -220,6 +240,48 @@ class PrefetchBudget(_Handle):
         f = np.empty(self.k + 1, np.int32)
         cov = _L().sv_prefetch_allocate(self._h, int(budget), f.ctypes.data)
         return f, float(cov)
+
+
+class FanoutPrefetcher:
+    """The fan-out pipeline around one NgramDrafter: while a request's draft
+    is being verified, ``prepare`` spends the budget (PrefetchBudget over the
+    recent outcomes) and drafts ahead for the outcomes it covers;
+    ``next_draft`` then serves the draft for the actual outcome (j, b) from
+    them (a hit) or drafts synchronously (a miss), and feeds the rank of b
+    among branch j's candidates back into the budget's window.  Drafts are
+    identical either way: prefetching only moves work off the critical path.
+    Requests are told apart by a caller-chosen key."""
+
+    def __init__(self, drafter: NgramDrafter, k: int = 16, budget: int = 16, fmax: int = 16, window: int = 256):
+        self.drafter, self.k, self.n_budget, self.fmax = drafter, int(k), int(budget), int(fmax)
+        self.budget = PrefetchBudget(self.k, self.fmax, window)
+        self.hits = self.misses = 0
+        self._pending = {}
+
+    def prepare(self, key, prompt_id: int, context, draft) -> float:
+        """Prefetch for request ``key`` (draft of at most k ids); returns the
+        expected hit rate the allocation predicts."""
+        ctx, d = [int(x) for x in context], [int(x) for x in draft]
+        if len(d) > self.k:
+            raise ValueError(f"draft of {len(d)} ids, the prefetcher was built for k = {self.k}")
+        f, coverage = self.budget.allocate(self.n_budget)
+        pre = self.drafter.prefetch(prompt_id, ctx, d, f[:len(d) + 1], self.k)
+        self._pending[key] = (prompt_id, ctx, d, pre)
+        return coverage
+
+    def next_draft(self, key, j: int, b: int):
+        """The next draft of request ``key`` after outcome (j, b), and
+        whether it came from the prefetch."""
+        prompt_id, ctx, d, pre = self._pending.pop(key)
+        branch = ctx + d[:j]
+        ranked = [int(x) for x in self.drafter.candidates(prompt_id, branch, self.fmax)]
+        self.budget.observe(j, ranked.index(b) if b in ranked else -1)
+        got = pre.get((int(j), int(b)))
+        if got is not None:
+            self.hits += 1
+            return got, True
+        self.misses += 1
+        return self.drafter.draft(prompt_id, branch + [int(b)], self.k), False
 
 
 class DraftLengthController(_Handle):
