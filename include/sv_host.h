@@ -49,6 +49,13 @@
  *  [ER-SWITCH] same page, section "三、聪明的开关": speculation is switched on
  *              only when the predicted speedup exceeds 1.05, and then stays on
  *              until the batch ends.
+ *  [ER-ROOF]   same section: the speedup comes from a roofline model (each
+ *              step bound by compute or by memory bandwidth; with many
+ *              sequences in flight the GPU is compute-bound and drafting plus
+ *              verifying loses, with few it is memory-bound and idle compute
+ *              makes verification cheap), calibrated once per model and
+ *              hardware by fitting its parameters to run times measured at
+ *              several batch sizes and sequence lengths.
  */
 #ifndef SV_HOST_H
 #define SV_HOST_H
@@ -251,6 +258,61 @@ SV_API double sv_block_efficiency(const int32_t *accept_len, int64_t n);
  * exceeded the threshold (1.05 on the page) since *state was set to 0, and
  * keeps returning 1 until the caller resets *state for the next batch. */
 SV_API int32_t sv_spec_switch(int32_t *state, double predicted_speedup, double threshold);
+
+/* ------------------------------------------------------------------------
+ * Roofline predictor behind the switch [ER-ROOF].
+ *
+ * A forward step of a decoder over B sequences, q new tokens each, with n
+ * tokens already cached per sequence, is either compute- or memory-bound:
+ *   flops(B, q, n) = 2 N B q + 4 L d B q n        (weights; attention over n)
+ *   bytes(B, q, n) = N w + 2 L h d_h e B n        (weights once; K and V read)
+ *   T(B, q, n)     = max(flops / pi, bytes / beta) + tau
+ * (a reading: the page names the two ceilings and a calibration, not the
+ * terms).  pi, beta and tau are calibrated once per model and machine from
+ * measured step times (sv_roofline_fit).  A speculative cycle with draft
+ * length k drafts k tokens one at a time and verifies k + 1 positions in one
+ * target step; with per-token acceptance alpha it yields
+ *   E = (1 - alpha^(k+1)) / (1 - alpha)  tokens   (E = k + 1 at alpha = 1),
+ * so the predicted speedup over plain decoding is
+ *   S = E T_t(B, 1, n) / (k T_d(B, 1, n) + T_t(B, k + 1, n)),
+ * which sv_spec_switch compares with 1.05.
+ */
+typedef struct {
+    double params;        /* N: weights */
+    double weight_bytes;  /* w: bytes per weight as stored (2 for bf16; ~0.56 for 4-bit with group scales) */
+    int32_t layers;       /* L */
+    int32_t width;        /* d: query heads x head dim */
+    int32_t kv_heads;     /* h */
+    int32_t head_dim;     /* d_h */
+    double kv_bytes;      /* e: bytes per cached K or V element */
+} sv_arch;
+
+typedef struct {
+    double flops_per_s;   /* pi */
+    double bytes_per_s;   /* beta */
+    double overhead_s;    /* tau */
+} sv_roofline;
+
+/* flops and bytes of one step; 0, or -1 on bad arguments (NULL, a negative
+ * or non-finite count, an architecture with a non-positive field). */
+SV_API int32_t sv_roofline_work(const sv_arch *a, double B, double q, double n, double *flops, double *bytes);
+/* T(B, q, n) in seconds; NaN on bad arguments. */
+SV_API double sv_roofline_time(const sv_arch *a, const sv_roofline *r, double B, double q, double n);
+/* Calibrate pi, beta, tau on m >= 3 measured steps (B[i], q[i], n[i],
+ * seconds[i] > 0): minimises the squared relative error
+ * sum_i ((T_i - seconds_i) / seconds_i)^2.  For fixed pi and beta the best
+ * tau >= 0 has a closed form; pi and beta are searched on a 41 x 41 log10
+ * grid from one decade below to three above the largest flops and bytes per
+ * measured second, then seven more times on a 10x finer grid spanning two
+ * steps of the previous one either side of its best point.  Writes the fit
+ * and, if rms_rel is not NULL,
+ * the root-mean-square relative error.  Returns 0, or -1 on bad arguments. */
+SV_API int32_t sv_roofline_fit(const sv_arch *a, int32_t m, const double *B, const double *q, const double *n,
+                               const double *seconds, sv_roofline *out, double *rms_rel);
+/* Predicted speedup S of speculative decoding (above); NaN on bad
+ * arguments (alpha outside [0, 1], k < 1, B <= 0, n < 0). */
+SV_API double sv_spec_speedup(const sv_arch *target, const sv_roofline *rt, const sv_arch *draft,
+                              const sv_roofline *rd, double B, int32_t k, double alpha, double n);
 
 /* ------------------------------------------------------------------------
  * Length-aware budgets [DAS-LEN].

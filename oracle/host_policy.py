@@ -243,3 +243,68 @@ def interleave_ranks(pred, world):
     for r, i in enumerate(order):
         ranks[i] = r % world
     return ranks
+
+
+# --------------------------------------------------------------------------
+# roofline predictor behind the switch (EfficientRollout article, section
+# "三、聪明的开关": each step bound by compute or by memory bandwidth,
+# calibrated on measured run times; the terms are this oracle's reading)
+
+def roofline_work(a, B, q, n):
+    """flops and bytes of one decoder step: every weight used twice per new
+    token (multiply and add) and read once; attention scores and values over
+    n cached positions (two width x n products per new token per layer); the
+    K and V cache read once."""
+    flops = 2.0 * a["params"] * B * q + 4.0 * a["layers"] * a["width"] * B * q * n
+    nbytes = a["params"] * a["weight_bytes"] + 2.0 * a["layers"] * a["kv_heads"] * a["head_dim"] * a["kv_bytes"] * B * n
+    return flops, nbytes
+
+
+def roofline_time(a, r, B, q, n):
+    f, m = roofline_work(a, B, q, n)
+    return max(f / r["flops_per_s"], m / r["bytes_per_s"]) + r["overhead_s"]
+
+
+def accepted_per_cycle(alpha, k):
+    """Expected tokens per draft-verify cycle with i.i.d. acceptance alpha:
+    the accepted prefix plus the one drawn token, summed term by term."""
+    return sum(alpha ** i for i in range(k + 1))
+
+
+def spec_speedup(target, rt, draft, rd, B, k, alpha, n):
+    cycle = k * roofline_time(draft, rd, B, 1, n) + roofline_time(target, rt, B, k + 1, n)
+    return accepted_per_cycle(alpha, k) * roofline_time(target, rt, B, 1, n) / cycle
+
+
+def roofline_fit(a, B, q, n, seconds, starts=12):
+    """Least squared relative error over (pi, beta, tau >= 0) by Nelder-Mead
+    from many starts in log space, tau by bounded scalar minimisation inside
+    (slow, and independent of the C++ grid search)."""
+    import numpy as np
+    from scipy import optimize
+    work = [roofline_work(a, b, qq, nn) for b, qq, nn in zip(B, q, n)]
+    t = [float(x) for x in seconds]
+
+    def err(lp, lb, tau):
+        pi, beta = 10.0 ** lp, 10.0 ** lb
+        return sum(((max(f / pi, m / beta) + tau - ti) / ti) ** 2 for (f, m), ti in zip(work, t))
+
+    def err2(x):
+        res = optimize.minimize_scalar(lambda tau: err(x[0], x[1], tau), bounds=(0.0, max(t)), method="bounded",
+                                       options={"xatol": 1e-15})
+        return min(res.fun, err(x[0], x[1], 0.0))
+
+    fr = max(f / ti for (f, _), ti in zip(work, t))
+    mr = max(m / ti for (_, m), ti in zip(work, t))
+    rng = np.random.default_rng(0)
+    best = None
+    for _ in range(starts):
+        x0 = [np.log10(fr) + rng.uniform(-1, 3), np.log10(mr) + rng.uniform(-1, 3)]
+        r = optimize.minimize(err2, x0, method="Nelder-Mead", options={"xatol": 1e-9, "fatol": 1e-16, "maxiter": 4000})
+        if best is None or r.fun < best.fun:
+            best = r
+    lp, lb = best.x
+    res = optimize.minimize_scalar(lambda tau: err(lp, lb, tau), bounds=(0.0, max(t)), method="bounded",
+                                   options={"xatol": 1e-15})
+    tau = res.x if res.fun < err(lp, lb, 0.0) else 0.0
+    return {"flops_per_s": 10.0 ** lp, "bytes_per_s": 10.0 ** lb, "overhead_s": tau}, err(lp, lb, tau)

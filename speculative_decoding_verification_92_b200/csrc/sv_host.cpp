@@ -687,3 +687,136 @@ int32_t sv_interleave_ranks(const double* predicted_len, int64_t n, int32_t worl
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Roofline predictor behind the switch.
+
+namespace {
+
+bool arch_ok(const sv_arch* a) {
+    return a && std::isfinite(a->params) && a->params > 0.0 && std::isfinite(a->weight_bytes) &&
+           a->weight_bytes > 0.0 && a->layers > 0 && a->width > 0 && a->kv_heads > 0 && a->head_dim > 0 &&
+           std::isfinite(a->kv_bytes) && a->kv_bytes > 0.0;
+}
+
+bool roofline_ok(const sv_roofline* r) {
+    return r && std::isfinite(r->flops_per_s) && r->flops_per_s > 0.0 && std::isfinite(r->bytes_per_s) &&
+           r->bytes_per_s > 0.0 && std::isfinite(r->overhead_s) && r->overhead_s >= 0.0;
+}
+
+bool count_ok(double x) { return std::isfinite(x) && x >= 0.0; }
+
+void step_work(const sv_arch& a, double B, double q, double n, double* flops, double* bytes) {
+    *flops = 2.0 * a.params * B * q + 4.0 * a.layers * static_cast<double>(a.width) * B * q * n;
+    *bytes = a.params * a.weight_bytes +
+             2.0 * a.layers * static_cast<double>(a.kv_heads) * a.head_dim * a.kv_bytes * B * n;
+}
+
+double step_time(const sv_roofline& r, double flops, double bytes) {
+    return std::max(flops / r.flops_per_s, bytes / r.bytes_per_s) + r.overhead_s;
+}
+
+// Sum of squared relative errors of the fit (pi, beta) with its best tau >= 0,
+// which is written to *tau: d/dtau sum ((m_i + tau - t_i) / t_i)^2 = 0 gives
+// tau = sum (t_i - m_i) / t_i^2 / sum 1 / t_i^2, clipped at 0 (the error is a
+// parabola in tau, so the clip is the constrained optimum).
+double fit_error(const std::vector<double>& F, const std::vector<double>& M, const double* t, double pi,
+                 double beta, double* tau) {
+    double num = 0.0, den = 0.0;
+    for (size_t i = 0; i < F.size(); ++i) {
+        const double m = std::max(F[i] / pi, M[i] / beta);
+        const double w = 1.0 / (t[i] * t[i]);
+        num += (t[i] - m) * w;
+        den += w;
+    }
+    const double tt = std::max(0.0, num / den);
+    double e = 0.0;
+    for (size_t i = 0; i < F.size(); ++i) {
+        const double d = (std::max(F[i] / pi, M[i] / beta) + tt - t[i]) / t[i];
+        e += d * d;
+    }
+    *tau = tt;
+    return e;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t sv_roofline_work(const sv_arch* a, double B, double q, double n, double* flops, double* bytes) {
+    if (!arch_ok(a) || !count_ok(B) || !count_ok(q) || !count_ok(n) || !flops || !bytes) return -1;
+    step_work(*a, B, q, n, flops, bytes);
+    return 0;
+}
+
+double sv_roofline_time(const sv_arch* a, const sv_roofline* r, double B, double q, double n) {
+    if (!arch_ok(a) || !roofline_ok(r) || !count_ok(B) || !count_ok(q) || !count_ok(n))
+        return std::numeric_limits<double>::quiet_NaN();
+    double F, M;
+    step_work(*a, B, q, n, &F, &M);
+    return step_time(*r, F, M);
+}
+
+int32_t sv_roofline_fit(const sv_arch* a, int32_t m, const double* B, const double* q, const double* n,
+                        const double* seconds, sv_roofline* out, double* rms_rel) {
+    if (!arch_ok(a) || m < 3 || !B || !q || !n || !seconds || !out) return -1;
+    try {
+        std::vector<double> F(static_cast<size_t>(m)), M(static_cast<size_t>(m));
+        double f_rate = 0.0, m_rate = 0.0;  // the largest flops and bytes per measured second
+        for (int32_t i = 0; i < m; ++i) {
+            if (!count_ok(B[i]) || !count_ok(q[i]) || !count_ok(n[i]) || !std::isfinite(seconds[i]) ||
+                !(seconds[i] > 0.0))
+                return -1;
+            step_work(*a, B[i], q[i], n[i], &F[i], &M[i]);
+            f_rate = std::max(f_rate, F[i] / seconds[i]);
+            m_rate = std::max(m_rate, M[i] / seconds[i]);
+        }
+        if (!(f_rate > 0.0) || !(m_rate > 0.0)) return -1;
+        // log10 grids: each rate lies at or above the fastest the data shows,
+        // so start from a decade below it to three above, 41 x 41 points;
+        // then re-grid +-2 steps around the best point, seven times
+        constexpr int kGrid = 41;
+        double lp0 = std::log10(f_rate) - 1.0, lb0 = std::log10(m_rate) - 1.0;
+        double step = 4.0 / (kGrid - 1);
+        double best_e = std::numeric_limits<double>::infinity(), best_lp = lp0, best_lb = lb0, best_tau = 0.0;
+        for (int round = 0; round < 8; ++round) {
+            const double cp = best_lp, cb = best_lb;
+            for (int i = 0; i < kGrid; ++i)
+                for (int j = 0; j < kGrid; ++j) {
+                    const double lp = round == 0 ? lp0 + i * step : cp + (i - kGrid / 2) * step;
+                    const double lb = round == 0 ? lb0 + j * step : cb + (j - kGrid / 2) * step;
+                    double tau;
+                    const double e = fit_error(F, M, seconds, std::pow(10.0, lp), std::pow(10.0, lb), &tau);
+                    if (e < best_e) {
+                        best_e = e;
+                        best_lp = lp;
+                        best_lb = lb;
+                        best_tau = tau;
+                    }
+                }
+            step = 4.0 * step / (kGrid - 1);  // the next grid spans +-2 steps of this one
+        }
+        out->flops_per_s = std::pow(10.0, best_lp);
+        out->bytes_per_s = std::pow(10.0, best_lb);
+        out->overhead_s = best_tau;
+        if (rms_rel) *rms_rel = std::sqrt(best_e / m);
+        return 0;
+    } catch (...) {
+        return -1;
+    }
+}
+
+double sv_spec_speedup(const sv_arch* target, const sv_roofline* rt, const sv_arch* draft, const sv_roofline* rd,
+                       double B, int32_t k, double alpha, double n) {
+    const double nan = std::numeric_limits<double>::quiet_NaN();
+    if (!arch_ok(target) || !roofline_ok(rt) || !arch_ok(draft) || !roofline_ok(rd) || !(B > 0.0) ||
+        !std::isfinite(B) || k < 1 || !(alpha >= 0.0 && alpha <= 1.0) || !count_ok(n))
+        return nan;
+    const double E = alpha >= 1.0 ? k + 1.0 : (1.0 - std::pow(alpha, k + 1.0)) / (1.0 - alpha);
+    const double t1 = sv_roofline_time(target, rt, B, 1.0, n);
+    const double tk = sv_roofline_time(target, rt, B, k + 1.0, n);
+    const double d1 = sv_roofline_time(draft, rd, B, 1.0, n);
+    return E * t1 / (k * d1 + tk);
+}
+
+}  // extern "C"

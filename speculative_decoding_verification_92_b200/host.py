@@ -35,6 +35,10 @@ _HOST_SIGNATURES = {
     "sv_prefetch_observe": (_I32, [_VP, _I32, _I32]),
     "sv_prefetch_estimates": (_I32, [_VP, _VP, _VP]),
     "sv_prefetch_allocate": (_F64, [_VP, _I32, _VP]),
+    "sv_roofline_work": (_I32, [_VP, _F64, _F64, _F64, _VP, _VP]),
+    "sv_roofline_time": (_F64, [_VP, _VP, _F64, _F64, _F64]),
+    "sv_roofline_fit": (_I32, [_VP, _I32, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "sv_spec_speedup": (_F64, [_VP, _VP, _VP, _VP, _F64, _I32, _F64, _F64]),
     "sv_ngram_prefetch": (_I32, [_VP, _I64, _VP, _I64, _VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP]),
     "sv_prefetch_find": (_I32, [_VP, _VP, _I32, _I32, _I32]),
     "sv_draft_len_create": (_VP, [_VP, _I32, _F64, _F64, _I32]),
@@ -330,3 +334,50 @@ def interleave_ranks(predicted_len, world_size: int):
     if _L().sv_interleave_ranks(x.ctypes.data, x.size, int(world_size), r.ctypes.data) != 0:
         raise ValueError("sv_interleave_ranks rejected its arguments")
     return r
+
+
+# ---------------------------------------------------------------------------
+# roofline predictor behind the speculation switch
+
+class Arch(ctypes.Structure):
+    """sv_arch: the decoder shape the roofline counts work from."""
+    _fields_ = [("params", ctypes.c_double), ("weight_bytes", ctypes.c_double), ("layers", ctypes.c_int32),
+                ("width", ctypes.c_int32), ("kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("kv_bytes", ctypes.c_double)]
+
+
+class Roofline(ctypes.Structure):
+    """sv_roofline: calibrated compute rate, bandwidth and per-step overhead."""
+    _fields_ = [("flops_per_s", ctypes.c_double), ("bytes_per_s", ctypes.c_double),
+                ("overhead_s", ctypes.c_double)]
+
+
+def roofline_work(arch: Arch, B, q, n):
+    """(flops, bytes) of one step over B sequences, q new tokens, n cached."""
+    f, b = ctypes.c_double(), ctypes.c_double()
+    if _L().sv_roofline_work(ctypes.byref(arch), float(B), float(q), float(n), ctypes.byref(f), ctypes.byref(b)):
+        raise ValueError("sv_roofline_work rejected its arguments")
+    return f.value, b.value
+
+
+def roofline_time(arch: Arch, roof: Roofline, B, q, n) -> float:
+    return float(_L().sv_roofline_time(ctypes.byref(arch), ctypes.byref(roof), float(B), float(q), float(n)))
+
+
+def roofline_fit(arch: Arch, B, q, n, seconds):
+    """Calibrate on measured steps; returns (Roofline, rms relative error)."""
+    cols = [np.ascontiguousarray(np.asarray(x, dtype=np.float64).reshape(-1)) for x in (B, q, n, seconds)]
+    m = cols[0].size
+    if any(c.size != m for c in cols):
+        raise ValueError("B, q, n and seconds must have the same length")
+    out, rms = Roofline(), ctypes.c_double()
+    if _L().sv_roofline_fit(ctypes.byref(arch), m, *(c.ctypes.data for c in cols), ctypes.byref(out),
+                            ctypes.byref(rms)):
+        raise ValueError("sv_roofline_fit rejected its arguments")
+    return out, rms.value
+
+
+def spec_speedup(target: Arch, rt: Roofline, draft: Arch, rd: Roofline, B, k: int, alpha: float, n) -> float:
+    """Predicted speedup of speculative decoding over plain decoding."""
+    return float(_L().sv_spec_speedup(ctypes.byref(target), ctypes.byref(rt), ctypes.byref(draft), ctypes.byref(rd),
+                                      float(B), int(k), float(alpha), float(n)))

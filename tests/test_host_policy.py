@@ -556,3 +556,129 @@ def test_prefetch_rejects_bad_arguments():
     assert lib.sv_prefetch_find(zero.ctypes.data, zero.ctypes.data, 4, 0, 0) == 0
     assert lib.sv_prefetch_find(zero.ctypes.data, zero.ctypes.data, 4, 1, 0) == -1
     assert lib.sv_prefetch_find(None, None, 4, 0, 0) == -1
+
+
+# ---------------------------------------------------------------------------
+# roofline predictor behind the speculation switch
+
+ARCH_8B = dict(params=8e9, weight_bytes=2.0, layers=32, width=4096, kv_heads=8, head_dim=128, kv_bytes=2.0)
+DRAFT_8B_W4 = dict(ARCH_8B, weight_bytes=0.5625)      # 4-bit weights with one fp16 scale per 32
+ROOF = dict(flops_per_s=1.5e15, bytes_per_s=6.0e12, overhead_s=30e-6)
+
+
+def calibration_grid():
+    B, q, n = [], [], []
+    for b in (1, 4, 16, 64, 256, 1024):
+        for qq in (1, 4, 9):
+            for nn in (128, 1024, 8192):
+                B.append(b)
+                q.append(qq)
+                n.append(nn)
+    return B, q, n
+
+
+def test_pin_roofline_work_against_explicit_tensors():
+    # A toy decoder built from explicit linear layers and attention matmuls:
+    # torch's flop counter (2 M N K per matmul) and the tensors' own sizes
+    # must give the oracle's flops and bytes.
+    import torch
+    from torch.utils.flop_counter import FlopCounterMode
+    L, d, h, dh, ff, Bt, qt, nt = 2, 64, 2, 16, 96, 3, 5, 7
+    torch.manual_seed(0)
+    layers = [dict(wq=torch.nn.Linear(d, d, bias=False), wk=torch.nn.Linear(d, h * dh, bias=False),
+                   wv=torch.nn.Linear(d, h * dh, bias=False), wo=torch.nn.Linear(d, d, bias=False),
+                   up=torch.nn.Linear(d, ff, bias=False), down=torch.nn.Linear(ff, d, bias=False))
+              for _ in range(L)]
+    params = sum(m.weight.numel() for lay in layers for m in lay.values())
+    heads = d // dh
+    kv = torch.zeros(L, 2, Bt, h, nt, dh)                 # the cached K and V
+    x = torch.randn(Bt, qt, d)
+    with torch.no_grad(), FlopCounterMode(display=False) as fc:
+        for li, lay in enumerate(layers):
+            Q = lay["wq"](x).view(Bt, qt, heads, dh).transpose(1, 2)          # [B, heads, q, dh]
+            lay["wk"](x)
+            lay["wv"](x)                                                     # new K, V (appended, not attended here)
+            K = kv[li, 0].repeat_interleave(heads // h, dim=1)               # [B, heads, n, dh]
+            V = kv[li, 1].repeat_interleave(heads // h, dim=1)
+            att = torch.matmul(Q, K.transpose(-1, -2))                       # scores over the n cached positions
+            o = torch.matmul(att, V).transpose(1, 2).reshape(Bt, qt, d)
+            x = lay["down"](lay["up"](lay["wo"](o)))
+    arch = dict(params=params, weight_bytes=2.0, layers=L, width=d, kv_heads=h, head_dim=dh, kv_bytes=2.0)
+    flops, nbytes = ho.roofline_work(arch, Bt, qt, nt)
+    assert flops == fc.get_total_flops()
+    assert nbytes == params * 2 + kv.numel() * 2
+    c = host.roofline_work(host.Arch(**arch), Bt, qt, nt)
+    assert c == (flops, nbytes)
+
+
+def test_pin_roofline_fit_recovers_known_parameters():
+    B, q, n = calibration_grid()
+    t = [ho.roofline_time(ARCH_8B, ROOF, *x) for x in zip(B, q, n)]
+    r, rms = host.roofline_fit(host.Arch(**ARCH_8B), B, q, n, t)
+    assert rms < 1e-6
+    assert abs(r.flops_per_s / ROOF["flops_per_s"] - 1) < 1e-6
+    assert abs(r.bytes_per_s / ROOF["bytes_per_s"] - 1) < 1e-6
+    assert abs(r.overhead_s - ROOF["overhead_s"]) < 1e-9
+
+
+def test_roofline_fit_parity_on_noisy_timings():
+    B, q, n = calibration_grid()
+    rng = np.random.default_rng(3)
+    t = np.array([ho.roofline_time(ARCH_8B, ROOF, *x) for x in zip(B, q, n)]) * np.exp(rng.normal(0, 0.03, len(B)))
+    r, rms = host.roofline_fit(host.Arch(**ARCH_8B), B, q, n, t)
+    ro, err = ho.roofline_fit(ARCH_8B, B, q, n, t)
+    assert rms ** 2 * len(B) <= err * (1 + 1e-9) + 1e-15        # at least as good an optimum
+    assert abs(r.flops_per_s / ro["flops_per_s"] - 1) < 1e-4
+    assert abs(r.bytes_per_s / ro["bytes_per_s"] - 1) < 1e-4
+    assert abs(r.overhead_s - ro["overhead_s"]) < 1e-8
+    assert 0.01 < rms < 0.05
+
+
+def test_pin_speedup_special_cases():
+    a, d = host.Arch(**ARCH_8B), host.Arch(**DRAFT_8B_W4)
+    r = host.Roofline(**ROOF)
+    for B, k, alpha, n in [(1, 5, 0.0, 512), (8, 7, 0.5, 4096), (64, 3, 0.9, 1024), (512, 11, 1.0, 2048)]:
+        want = ho.spec_speedup(ARCH_8B, ROOF, DRAFT_8B_W4, ROOF, B, k, alpha, n)
+        assert abs(host.spec_speedup(a, r, d, r, B, k, alpha, n) / want - 1) < 1e-12
+    # alpha = 0: one token per cycle, so drafting can only lose
+    assert host.spec_speedup(a, r, d, r, 4, 5, 0.0, 512) < 1
+    # a free draft on a memory-bound target: the cycle costs one plain step and
+    # yields E = (1 - alpha^(k+1)) / (1 - alpha) tokens
+    tiny = host.Arch(params=1.0, weight_bytes=1e-9, layers=1, width=1, kv_heads=1, head_dim=1, kv_bytes=1e-12)
+    free = host.Roofline(flops_per_s=1e30, bytes_per_s=1e30, overhead_s=0.0)
+    r0 = host.Roofline(flops_per_s=1.5e15, bytes_per_s=6.0e12, overhead_s=0.0)
+    for alpha, k in [(0.5, 4), (0.8, 7), (1.0, 5)]:
+        E = k + 1 if alpha == 1 else (1 - alpha ** (k + 1)) / (1 - alpha)
+        assert abs(host.spec_speedup(a, r0, tiny, free, 1, k, alpha, 64) / E - 1) < 1e-3
+
+
+def test_pin_switch_regions_follow_the_batch():
+    # the page: with many sequences in flight the GPU is compute-bound and
+    # speculation loses; as the batch drains it becomes memory-bound and wins,
+    # and the switch, once on, stays on
+    a, d, r = host.Arch(**ARCH_8B), host.Arch(**DRAFT_8B_W4), host.Roofline(**ROOF)
+    sizes = [1024, 768, 512, 384, 256, 192, 128, 96, 64, 48, 32, 16, 8, 4, 2, 1]
+    s = [host.spec_speedup(a, r, d, r, B, 5, 0.9, 2048) for B in sizes]
+    assert s[0] < 1 and s[-1] > 1.05
+    assert all(x <= y + 1e-12 for x, y in zip(s, s[1:]))       # shrinking batch, rising speedup
+    state = [0]
+    on = [host.spec_switch(state, x) for x in s]
+    first = on.index(1)
+    assert s[first] > 1.05 and s[first - 1] <= 1.05 and all(on[first:])
+    assert ho.spec_switch(s) == on
+
+
+def test_roofline_rejects_bad_arguments():
+    a = host.Arch(**ARCH_8B)
+    with pytest.raises(ValueError):
+        host.roofline_work(host.Arch(**dict(ARCH_8B, layers=0)), 1, 1, 1)
+    with pytest.raises(ValueError):
+        host.roofline_work(a, -1, 1, 1)
+    with pytest.raises(ValueError):
+        host.roofline_fit(a, [1, 2], [1, 1], [0, 0], [1e-3, 2e-3])            # fewer than 3 steps
+    with pytest.raises(ValueError):
+        host.roofline_fit(a, [1, 2, 3], [1, 1, 1], [0, 0, 0], [1e-3, 0.0, 2e-3])
+    r = host.Roofline(**ROOF)
+    assert math.isnan(host.spec_speedup(a, r, a, r, 4, 0, 0.5, 10))
+    assert math.isnan(host.spec_speedup(a, r, a, r, 4, 5, 1.5, 10))
+    assert math.isnan(host.roofline_time(a, host.Roofline(0.0, 1.0, 0.0), 1, 1, 1))
