@@ -378,6 +378,16 @@ def test_batched_drafting_matches_the_oracle_for_every_thread_count(which):
     # without caps every request may use k_max
     tok2, lens2 = c.draft_batch(ids, ctxs, k_max)
     assert np.all(lens2 >= lens)
+    # a batch large enough for several threads (at least 512 requests each)
+    big = rng.integers(0, 8, size=2100)
+    big_ctx = [ctxs[i % B] for i in range(big.size)]
+    one = c.draft_batch(big, big_ctx, k_max, n_threads=1)
+    for nt in (2, 4, 0):
+        many = c.draft_batch(big, big_ctx, k_max, n_threads=nt)
+        assert np.array_equal(many[0], one[0]) and np.array_equal(many[1], one[1])
+    for i in range(0, big.size, 97):
+        want = o.draft(int(big[i]), big_ctx[i], k_max)
+        assert list(one[0][i, :one[1][i]]) == want
 
 
 def test_batched_drafting_rejects_bad_arguments():
