@@ -2,8 +2,10 @@
 
 The work runs in ``libspecverify.so`` (CUDA kernels for sm_100a, declared in
 ``include/spec_verify.h``).  This module is a thin ctypes binding: it checks
-tensor dtypes / devices, passes raw pointers and the current CUDA stream, and
-turns status codes into exceptions.  PyTorch is used only for device memory
+tensor shapes, dtypes and devices, passes raw pointers and the current CUDA
+stream, and turns status codes into exceptions.  ``host`` binds the host-side
+drafters and schedulers of ``include/sv_host.h``; ``graph`` replays a whole
+step as one CUDA graph.  PyTorch is used only for device memory
 and streams.  There is no CPU fallback: without the built library every call
 raises.
 
