@@ -40,21 +40,35 @@ uint64_t hash_tokens(const int32_t* t, int64_t n) {
 
 // ===========================================================================
 // Per-prompt n-gram drafter.
+//
+// One index per prompt maps every n-gram (n = 1..max_n) of its retained
+// rollouts to its occurrences, each stored as (rollout sequence number,
+// continuation start) in 8 bytes.  Rollouts get consecutive sequence numbers
+// in the order they are added, so every occurrence list is sorted oldest
+// first and the most recent occurrence is found from its back; a lookup costs
+// one hash probe per n whatever the number of rollouts.  Evicting a step's
+// rollouts cuts the same prefix off every list.
 
 struct sv_ngram {
     struct Rollout {
         int64_t step;
         std::vector<int32_t> tok;
-        // key of the n-gram tok[p-n .. p) (n = 1..max_n) -> every p, ascending;
-        // p is the position right after the n-gram (where a continuation starts)
-        std::unordered_map<uint64_t, std::vector<int32_t>> ends;
+    };
+    struct Occ {
+        int32_t seq;  // rollout sequence number within the prompt
+        int32_t p;    // continuation start: the n-gram is tok[p-n .. p), tok[p] exists
+    };
+    struct Prompt {
+        std::deque<Rollout> rollouts;  // oldest first; rollouts[i] has sequence number first_seq + i
+        int32_t first_seq = 0;
+        std::unordered_map<uint64_t, std::vector<Occ>> index;  // n-gram key -> occurrences, oldest first
+        const Rollout& rollout(int32_t seq) const { return rollouts[static_cast<size_t>(seq - first_seq)]; }
     };
     int32_t max_n = 6;
     int32_t window = 4;
     int64_t step = 0;
     bool started = false;
-    // per prompt, oldest first (so newest = back)
-    std::unordered_map<int64_t, std::deque<Rollout>> prompts;
+    std::unordered_map<int64_t, Prompt> prompts;
 };
 
 namespace {
@@ -64,35 +78,31 @@ struct Occurrence {
     int64_t p = -1;  // continuation start
 };
 
-// The last n context tokens followed by at least one token in rollout r:
-// the latest such position, or -1.
-int64_t latest_in(const sv_ngram::Rollout& r, const int32_t* key, int32_t n, uint64_t h) {
-    auto it = r.ends.find(h);
-    if (it == r.ends.end()) return -1;
-    const std::vector<int32_t>& ps = it->second;
-    for (auto q = ps.rbegin(); q != ps.rend(); ++q) {
-        const int64_t p = *q;
-        if (p >= static_cast<int64_t>(r.tok.size())) continue;  // nothing follows
-        if (std::memcmp(r.tok.data() + p - n, key, sizeof(int32_t) * n) == 0) return p;
-    }
-    return -1;
+// Whether occurrence q of the list under key's hash really is the n-gram
+// key[0..n) (a hash collision, with another n-gram or another n, is not).
+bool occ_matches(const sv_ngram::Prompt& pr, const sv_ngram::Occ& q, const int32_t* key, int32_t n) {
+    if (q.p < n) return false;
+    const sv_ngram::Rollout& r = pr.rollout(q.seq);
+    return std::memcmp(r.tok.data() + q.p - n, key, sizeof(int32_t) * n) == 0;
 }
 
-// Longest n with an occurrence; fills the most recent occurrence.
-int32_t longest_match(const sv_ngram& t, const std::deque<sv_ngram::Rollout>& rs, const int32_t* ctx,
-                      int64_t n_ctx, Occurrence* occ) {
+// Longest n whose last n context tokens occur followed by a token; fills the
+// most recent occurrence (latest step, then latest rollout, then latest
+// position: the back of the sorted list).
+int32_t longest_match(const sv_ngram& t, const sv_ngram::Prompt& pr, const int32_t* ctx, int64_t n_ctx,
+                      Occurrence* occ) {
     const int32_t top = static_cast<int32_t>(std::min<int64_t>(t.max_n, n_ctx));
     for (int32_t n = top; n >= 1; --n) {
         const int32_t* key = ctx + n_ctx - n;
-        const uint64_t h = hash_tokens(key, n);
-        for (auto r = rs.rbegin(); r != rs.rend(); ++r) {
-            const int64_t p = latest_in(*r, key, n, h);
-            if (p >= 0) {
-                occ->r = &*r;
-                occ->p = p;
+        auto it = pr.index.find(hash_tokens(key, n));
+        if (it == pr.index.end()) continue;
+        const std::vector<sv_ngram::Occ>& v = it->second;
+        for (auto q = v.rbegin(); q != v.rend(); ++q)
+            if (occ_matches(pr, *q, key, n)) {
+                occ->r = &pr.rollout(q->seq);
+                occ->p = q->p;
                 return n;
             }
-        }
     }
     return 0;
 }
@@ -117,24 +127,48 @@ void sv_ngram_begin_step(sv_ngram* t) {
     if (t->started) ++t->step;
     t->started = true;
     for (auto it = t->prompts.begin(); it != t->prompts.end();) {
-        auto& rs = it->second;
-        while (!rs.empty() && rs.front().step <= t->step - t->window) rs.pop_front();
-        if (rs.empty()) it = t->prompts.erase(it);
-        else ++it;
+        sv_ngram::Prompt& pr = it->second;
+        const int32_t before = pr.first_seq;
+        while (!pr.rollouts.empty() && pr.rollouts.front().step <= t->step - t->window) {
+            pr.rollouts.pop_front();
+            ++pr.first_seq;
+        }
+        if (pr.rollouts.empty()) {
+            it = t->prompts.erase(it);
+            continue;
+        }
+        if (pr.first_seq != before) {
+            // the evicted rollouts are the oldest: a prefix of every list
+            for (auto e = pr.index.begin(); e != pr.index.end();) {
+                std::vector<sv_ngram::Occ>& v = e->second;
+                auto keep = std::lower_bound(v.begin(), v.end(), pr.first_seq,
+                                             [](const sv_ngram::Occ& q, int32_t s) { return q.seq < s; });
+                v.erase(v.begin(), keep);
+                if (v.empty()) e = pr.index.erase(e);
+                else ++e;
+            }
+        }
+        ++it;
     }
 }
 
 int32_t sv_ngram_add(sv_ngram* t, int64_t prompt_id, const int32_t* tokens, int64_t n) {
     if (!t || n < 0 || (n > 0 && !tokens) || n > std::numeric_limits<int32_t>::max()) return -1;
     if (!t->started) sv_ngram_begin_step(t);
-    sv_ngram::Rollout r;
-    r.step = t->step;
-    r.tok.assign(tokens, tokens + n);
-    for (int64_t p = 1; p <= n; ++p)
-        for (int32_t k = 1; k <= t->max_n && k <= p; ++k)
-            r.ends[hash_tokens(tokens + p - k, k)].push_back(static_cast<int32_t>(p));
-    t->prompts[prompt_id].push_back(std::move(r));
-    return 0;
+    try {
+        sv_ngram::Prompt& pr = t->prompts[prompt_id];
+        if (pr.first_seq + static_cast<int64_t>(pr.rollouts.size()) >= std::numeric_limits<int32_t>::max())
+            return -1;
+        const int32_t seq = pr.first_seq + static_cast<int32_t>(pr.rollouts.size());
+        pr.rollouts.push_back(sv_ngram::Rollout{t->step, std::vector<int32_t>(tokens, tokens + n)});
+        // n-grams that some token follows: continuation starts p = 1 .. n-1
+        for (int64_t p = 1; p < n; ++p)
+            for (int32_t k = 1; k <= t->max_n && k <= p; ++k)
+                pr.index[hash_tokens(tokens + p - k, k)].push_back({seq, static_cast<int32_t>(p)});
+        return 0;
+    } catch (...) {
+        return -1;
+    }
 }
 
 int32_t sv_ngram_draft(const sv_ngram* t, int64_t prompt_id, const int32_t* context, int64_t n, int32_t k,
@@ -155,26 +189,22 @@ int32_t sv_ngram_candidates(const sv_ngram* t, int64_t prompt_id, const int32_t*
     if (!t || n < 0 || (n > 0 && !context) || f < 0 || (f > 0 && !out)) return -1;
     auto it = t->prompts.find(prompt_id);
     if (it == t->prompts.end() || n == 0 || f == 0) return 0;
+    const sv_ngram::Prompt& pr = it->second;
     Occurrence occ;
-    const int32_t nm = longest_match(*t, it->second, context, n, &occ);
+    const int32_t nm = longest_match(*t, pr, context, n, &occ);
     if (nm == 0) return 0;
     // every occurrence of the matched n-gram, newest first: count followers
     // and remember the order of their most recent occurrence
     const int32_t* key = context + n - nm;
-    const uint64_t h = hash_tokens(key, nm);
     struct Cand { int32_t tok; int64_t count; int64_t first_seen; };
-    std::vector<Cand> cands;
-    std::unordered_map<int32_t, size_t> slot;
-    int64_t order = 0;
-    const auto& rs = it->second;
-    for (auto r = rs.rbegin(); r != rs.rend(); ++r) {
-        auto e = r->ends.find(h);
-        if (e == r->ends.end()) continue;
-        for (auto q = e->second.rbegin(); q != e->second.rend(); ++q) {
-            const int64_t p = *q;
-            if (p >= static_cast<int64_t>(r->tok.size())) continue;
-            if (std::memcmp(r->tok.data() + p - nm, key, sizeof(int32_t) * nm) != 0) continue;
-            const int32_t nxt = r->tok[p];
+    try {
+        std::vector<Cand> cands;
+        std::unordered_map<int32_t, size_t> slot;
+        int64_t order = 0;
+        const std::vector<sv_ngram::Occ>& v = pr.index.find(hash_tokens(key, nm))->second;
+        for (auto q = v.rbegin(); q != v.rend(); ++q) {
+            if (!occ_matches(pr, *q, key, nm)) continue;
+            const int32_t nxt = pr.rollout(q->seq).tok[static_cast<size_t>(q->p)];
             auto s = slot.find(nxt);
             if (s == slot.end()) {
                 slot.emplace(nxt, cands.size());
@@ -184,19 +214,21 @@ int32_t sv_ngram_candidates(const sv_ngram* t, int64_t prompt_id, const int32_t*
             }
             ++order;
         }
+        std::stable_sort(cands.begin(), cands.end(), [](const Cand& a, const Cand& b) {
+            return a.count != b.count ? a.count > b.count : a.first_seen < b.first_seen;
+        });
+        const int32_t m = static_cast<int32_t>(std::min<size_t>(f, cands.size()));
+        for (int32_t i = 0; i < m; ++i) out[i] = cands[i].tok;
+        return m;
+    } catch (...) {
+        return -1;
     }
-    std::stable_sort(cands.begin(), cands.end(), [](const Cand& a, const Cand& b) {
-        return a.count != b.count ? a.count > b.count : a.first_seen < b.first_seen;
-    });
-    const int32_t m = static_cast<int32_t>(std::min<size_t>(f, cands.size()));
-    for (int32_t i = 0; i < m; ++i) out[i] = cands[i].tok;
-    return m;
 }
 
 int64_t sv_ngram_rollouts(const sv_ngram* t) {
     if (!t) return -1;
     int64_t n = 0;
-    for (const auto& kv : t->prompts) n += static_cast<int64_t>(kv.second.size());
+    for (const auto& kv : t->prompts) n += static_cast<int64_t>(kv.second.rollouts.size());
     return n;
 }
 
@@ -204,7 +236,7 @@ int64_t sv_ngram_tokens(const sv_ngram* t) {
     if (!t) return -1;
     int64_t n = 0;
     for (const auto& kv : t->prompts)
-        for (const auto& r : kv.second) n += static_cast<int64_t>(r.tok.size());
+        for (const auto& r : kv.second.rollouts) n += static_cast<int64_t>(r.tok.size());
     return n;
 }
 
