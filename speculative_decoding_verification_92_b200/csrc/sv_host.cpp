@@ -244,15 +244,29 @@ int64_t sv_ngram_tokens(const sv_ngram* t) {
 
 // ===========================================================================
 // Suffix drafter with frequency scoring.
+//
+// Every distinct context (the d <= max_depth tokens before some position of a
+// trajectory) is one 32-byte entry that points at its first occurrence in a
+// trajectory instead of copying it, and keeps its first follower inline; the
+// rare further followers go to a side list.  A hash of the context selects a
+// chain of entries; a context is confirmed by comparing its tokens.
 
 struct sv_suffix {
-    struct Context {
-        std::vector<int32_t> ctx;                    // the context tokens
-        std::unordered_map<int32_t, int64_t> next;   // follower -> count
+    struct Entry {
+        int32_t traj;   // trajectory holding the context's first occurrence
+        int32_t end;    // the context is that trajectory's tokens [end - d, end)
+        int32_t d;
+        int32_t chain;  // next entry under the same hash, or -1
+        int64_t cnt0;   // count of the first follower seen
+        int32_t tok0;   // that follower
+        int32_t more;   // index of the list of further followers, or -1
     };
     struct Problem {
-        std::unordered_map<int64_t, std::vector<int32_t>> seqs;
-        std::unordered_map<uint64_t, std::vector<Context>> table;  // hash of ctx -> contexts
+        std::unordered_map<int64_t, int32_t> slot;                    // seq_id -> trajectory index
+        std::vector<std::vector<int32_t>> trajs;
+        std::unordered_map<uint64_t, int32_t> head;                   // context hash -> first entry
+        std::vector<Entry> entries;
+        std::vector<std::vector<std::pair<int32_t, int64_t>>> extra;  // followers beyond the first
     };
     int32_t max_depth = 8;
     std::unordered_map<int64_t, Problem> problems;
@@ -260,35 +274,49 @@ struct sv_suffix {
 
 namespace {
 
-const sv_suffix::Context* find_context(const sv_suffix::Problem& pb, const int32_t* c, int32_t d) {
-    auto it = pb.table.find(hash_tokens(c, d));
-    if (it == pb.table.end()) return nullptr;
-    for (const auto& e : it->second)
-        if (static_cast<int32_t>(e.ctx.size()) == d && std::memcmp(e.ctx.data(), c, sizeof(int32_t) * d) == 0)
+const sv_suffix::Entry* find_context(const sv_suffix::Problem& pb, const int32_t* c, int32_t d) {
+    auto it = pb.head.find(hash_tokens(c, d));
+    if (it == pb.head.end()) return nullptr;
+    for (int32_t i = it->second; i >= 0; i = pb.entries[static_cast<size_t>(i)].chain) {
+        const sv_suffix::Entry& e = pb.entries[static_cast<size_t>(i)];
+        if (e.d == d &&
+            std::memcmp(pb.trajs[static_cast<size_t>(e.traj)].data() + e.end - d, c, sizeof(int32_t) * d) == 0)
             return &e;
+    }
     return nullptr;
 }
 
 // Longest d <= max_depth with a count table for the last d tokens of c[0..n).
-const sv_suffix::Context* longest_context(const sv_suffix& t, const sv_suffix::Problem& pb, const int32_t* c,
-                                          int64_t n) {
+const sv_suffix::Entry* longest_context(const sv_suffix& t, const sv_suffix::Problem& pb, const int32_t* c,
+                                        int64_t n) {
     const int32_t top = static_cast<int32_t>(std::min<int64_t>(t.max_depth, n));
     for (int32_t d = top; d >= 1; --d) {
-        const sv_suffix::Context* e = find_context(pb, c + n - d, d);
+        const sv_suffix::Entry* e = find_context(pb, c + n - d, d);
         if (e) return e;
     }
     return nullptr;
 }
 
+// Every follower of e with its count, in no particular order.
+std::vector<std::pair<int32_t, int64_t>> followers(const sv_suffix::Problem& pb, const sv_suffix::Entry& e) {
+    std::vector<std::pair<int32_t, int64_t>> c{{e.tok0, e.cnt0}};
+    if (e.more >= 0) {
+        const auto& x = pb.extra[static_cast<size_t>(e.more)];
+        c.insert(c.end(), x.begin(), x.end());
+    }
+    return c;
+}
+
 // Most frequent follower, ties to the lowest id.
-int32_t top_follower(const sv_suffix::Context& e) {
-    int32_t best = 0;
-    int64_t best_n = -1;
-    for (const auto& kv : e.next)
-        if (kv.second > best_n || (kv.second == best_n && kv.first < best)) {
-            best = kv.first;
-            best_n = kv.second;
-        }
+int32_t top_follower(const sv_suffix::Problem& pb, const sv_suffix::Entry& e) {
+    int32_t best = e.tok0;
+    int64_t best_n = e.cnt0;
+    if (e.more >= 0)
+        for (const auto& kv : pb.extra[static_cast<size_t>(e.more)])
+            if (kv.second > best_n || (kv.second == best_n && kv.first < best)) {
+                best = kv.first;
+                best_n = kv.second;
+            }
     return best;
 }
 
@@ -312,29 +340,51 @@ void sv_suffix_clear(sv_suffix* t) {
 
 int32_t sv_suffix_append(sv_suffix* t, int64_t problem_id, int64_t seq_id, const int32_t* tokens, int64_t m) {
     if (!t || m < 0 || (m > 0 && !tokens)) return -1;
-    sv_suffix::Problem& pb = t->problems[problem_id];
-    std::vector<int32_t>& seq = pb.seqs[seq_id];
-    for (int64_t i = 0; i < m; ++i) {
-        const int32_t tok = tokens[i];
-        const int64_t n = static_cast<int64_t>(seq.size());
-        for (int32_t d = 1; d <= t->max_depth && d <= n; ++d) {
-            const int32_t* c = seq.data() + n - d;
-            auto& bucket = pb.table[hash_tokens(c, d)];
-            sv_suffix::Context* e = nullptr;
-            for (auto& x : bucket)
-                if (static_cast<int32_t>(x.ctx.size()) == d && std::memcmp(x.ctx.data(), c, sizeof(int32_t) * d) == 0) {
-                    e = &x;
-                    break;
-                }
-            if (!e) {
-                bucket.push_back(sv_suffix::Context{std::vector<int32_t>(c, c + d), {}});
-                e = &bucket.back();
-            }
-            ++e->next[tok];
+    try {
+        sv_suffix::Problem& pb = t->problems[problem_id];
+        auto sl = pb.slot.find(seq_id);
+        if (sl == pb.slot.end()) {
+            if (pb.trajs.size() >= static_cast<size_t>(std::numeric_limits<int32_t>::max())) return -1;
+            sl = pb.slot.emplace(seq_id, static_cast<int32_t>(pb.trajs.size())).first;
+            pb.trajs.emplace_back();
         }
-        seq.push_back(tok);
+        const int32_t ti = sl->second;
+        std::vector<int32_t>& seq = pb.trajs[static_cast<size_t>(ti)];
+        if (static_cast<int64_t>(seq.size()) + m > std::numeric_limits<int32_t>::max()) return -1;
+        for (int64_t i = 0; i < m; ++i) {
+            const int32_t tok = tokens[i];
+            const int32_t n = static_cast<int32_t>(seq.size());
+            for (int32_t d = 1; d <= t->max_depth && d <= n; ++d) {
+                const int32_t* c = seq.data() + n - d;
+                const sv_suffix::Entry* found = find_context(pb, c, d);
+                if (!found) {
+                    if (pb.entries.size() >= static_cast<size_t>(std::numeric_limits<int32_t>::max())) return -1;
+                    const int32_t idx = static_cast<int32_t>(pb.entries.size());
+                    int32_t& h = pb.head.try_emplace(hash_tokens(c, d), -1).first->second;
+                    pb.entries.push_back(sv_suffix::Entry{ti, n, d, h, 1, tok, -1});
+                    h = idx;
+                    continue;
+                }
+                sv_suffix::Entry& e = pb.entries[static_cast<size_t>(found - pb.entries.data())];
+                if (e.tok0 == tok) {
+                    ++e.cnt0;
+                    continue;
+                }
+                if (e.more < 0) {
+                    e.more = static_cast<int32_t>(pb.extra.size());
+                    pb.extra.emplace_back();
+                }
+                auto& x = pb.extra[static_cast<size_t>(e.more)];
+                auto f = std::find_if(x.begin(), x.end(), [tok](const auto& kv) { return kv.first == tok; });
+                if (f == x.end()) x.emplace_back(tok, 1);
+                else ++f->second;
+            }
+            seq.push_back(tok);
+        }
+        return 0;
+    } catch (...) {
+        return -1;
     }
-    return 0;
 }
 
 int32_t sv_suffix_draft(const sv_suffix* t, int64_t problem_id, const int32_t* context, int64_t n, int32_t k,
@@ -342,18 +392,23 @@ int32_t sv_suffix_draft(const sv_suffix* t, int64_t problem_id, const int32_t* c
     if (!t || n < 0 || (n > 0 && !context) || k < 0 || (k > 0 && !out)) return -1;
     auto it = t->problems.find(problem_id);
     if (it == t->problems.end() || k == 0) return 0;
-    // the draft extends the context: keep the last max_depth tokens of both
-    std::vector<int32_t> ctx(context + std::max<int64_t>(0, n - t->max_depth), context + n);
-    int32_t m = 0;
-    while (m < k) {
-        const sv_suffix::Context* e = longest_context(*t, it->second, ctx.data(), static_cast<int64_t>(ctx.size()));
-        if (!e) break;
-        const int32_t tok = top_follower(*e);
-        out[m++] = tok;
-        ctx.push_back(tok);
-        if (static_cast<int32_t>(ctx.size()) > t->max_depth) ctx.erase(ctx.begin());
+    try {
+        // the draft extends the context: keep the last max_depth tokens of both
+        std::vector<int32_t> ctx(context + std::max<int64_t>(0, n - t->max_depth), context + n);
+        int32_t m = 0;
+        while (m < k) {
+            const sv_suffix::Entry* e =
+                longest_context(*t, it->second, ctx.data(), static_cast<int64_t>(ctx.size()));
+            if (!e) break;
+            const int32_t tok = top_follower(it->second, *e);
+            out[m++] = tok;
+            ctx.push_back(tok);
+            if (static_cast<int32_t>(ctx.size()) > t->max_depth) ctx.erase(ctx.begin());
+        }
+        return m;
+    } catch (...) {
+        return -1;
     }
-    return m;
 }
 
 int32_t sv_suffix_candidates(const sv_suffix* t, int64_t problem_id, const int32_t* context, int64_t n, int32_t f,
@@ -361,15 +416,19 @@ int32_t sv_suffix_candidates(const sv_suffix* t, int64_t problem_id, const int32
     if (!t || n < 0 || (n > 0 && !context) || f < 0 || (f > 0 && !out)) return -1;
     auto it = t->problems.find(problem_id);
     if (it == t->problems.end() || f == 0) return 0;
-    const sv_suffix::Context* e = longest_context(*t, it->second, context, n);
+    const sv_suffix::Entry* e = longest_context(*t, it->second, context, n);
     if (!e) return 0;
-    std::vector<std::pair<int32_t, int64_t>> c(e->next.begin(), e->next.end());
-    std::sort(c.begin(), c.end(), [](const auto& a, const auto& b) {
-        return a.second != b.second ? a.second > b.second : a.first < b.first;
-    });
-    const int32_t m = static_cast<int32_t>(std::min<size_t>(f, c.size()));
-    for (int32_t i = 0; i < m; ++i) out[i] = c[i].first;
-    return m;
+    try {
+        std::vector<std::pair<int32_t, int64_t>> c = followers(it->second, *e);
+        std::sort(c.begin(), c.end(), [](const auto& a, const auto& b) {
+            return a.second != b.second ? a.second > b.second : a.first < b.first;
+        });
+        const int32_t m = static_cast<int32_t>(std::min<size_t>(f, c.size()));
+        for (int32_t i = 0; i < m; ++i) out[i] = c[i].first;
+        return m;
+    } catch (...) {
+        return -1;
+    }
 }
 
 }  // extern "C"
