@@ -70,14 +70,28 @@ def _tok(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a, dtype=np.int32).reshape(-1))
 
 
-def _draft_batch(fn, h, ids, contexts, k_max, max_lens, n_threads):
+def _tail(a, n: int) -> np.ndarray:
+    """The last n tokens of a context (a lookup never reads further back);
+    sliced before conversion when the context supports it."""
+    try:
+        if len(a) > n:
+            a = a[-n:]
+    except TypeError:
+        pass
+    return _tok(a)[-n:]
+
+
+def _draft_batch(fn, h, ids, contexts, k_max, max_lens, n_threads, tail):
     """Shared marshalling of the batched drafting calls: returns the
     drafted-id array [B, k_max] (-1 padded) and the lengths [B], both int32,
-    in the layout spec_verify takes as draft_tokens / draft_lens."""
+    in the layout spec_verify takes as draft_tokens / draft_lens.  Only the
+    last ``tail`` tokens of each context can take part in a match, so only
+    those are passed."""
     ids = np.ascontiguousarray(np.asarray(ids, dtype=np.int64).reshape(-1))
     B = ids.size
     if len(contexts) != B:
         raise ValueError(f"{B} ids but {len(contexts)} contexts")
+    contexts = [c[-tail:] if len(c) > tail else c for c in contexts]
     off = np.zeros(B + 1, np.int64)
     np.cumsum(np.fromiter((len(c) for c in contexts), np.int64, count=B), out=off[1:])
     # one concatenation (and one conversion to int32) for the whole batch
@@ -127,6 +141,7 @@ class NgramDrafter(_Handle):
 
     def __init__(self, max_n: int = 6, window: int = 4):
         super().__init__(_L().sv_ngram_create(int(max_n), int(window)))
+        self.max_n = int(max_n)     # the longest context tail a lookup can use
 
     def begin_step(self):
         _L().sv_ngram_begin_step(self._h)
@@ -137,7 +152,7 @@ class NgramDrafter(_Handle):
             raise ValueError("sv_ngram_add rejected its arguments")
 
     def draft(self, prompt_id: int, context, k: int = 16) -> np.ndarray:
-        c = _tok(context)
+        c = _tail(context, self.max_n)
         out = np.empty(max(int(k), 1), np.int32)
         n = _L().sv_ngram_draft(self._h, int(prompt_id), c.ctypes.data, c.size, int(k), out.ctypes.data)
         if n < 0:
@@ -148,7 +163,7 @@ class NgramDrafter(_Handle):
         """Next drafts for the verification outcomes that the allocation
         ``f`` (one entry per branch j = 0..len(draft)) covers, drafted before
         the outcome is known: ``{(j, b): ids}`` (sv_ngram_prefetch)."""
-        c, d = _tok(context), _tok(draft)
+        c, d = _tail(context, self.max_n), _tok(draft)
         fa = np.ascontiguousarray(np.asarray(f, dtype=np.int32).reshape(-1))
         if fa.size != d.size + 1:
             raise ValueError(f"f needs {d.size + 1} entries (branches j = 0..{d.size}), got {fa.size}")
@@ -167,10 +182,11 @@ class NgramDrafter(_Handle):
         draft_lens [B])`` int32, -1 padded, ready for spec_verify without
         draft logits.  ``max_lens`` caps each request (controller length or
         budget); ``n_threads`` 0 uses the hardware threads."""
-        return _draft_batch(_L().sv_ngram_draft_batch, self._h, prompt_ids, contexts, k_max, max_lens, n_threads)
+        return _draft_batch(_L().sv_ngram_draft_batch, self._h, prompt_ids, contexts, k_max, max_lens, n_threads,
+                            self.max_n)
 
     def candidates(self, prompt_id: int, context, f: int) -> np.ndarray:
-        c = _tok(context)
+        c = _tail(context, self.max_n)
         out = np.empty(max(int(f), 1), np.int32)
         n = _L().sv_ngram_candidates(self._h, int(prompt_id), c.ctypes.data, c.size, int(f), out.ctypes.data)
         if n < 0:
@@ -192,6 +208,7 @@ class SuffixDrafter(_Handle):
 
     def __init__(self, max_depth: int = 8):
         super().__init__(_L().sv_suffix_create(int(max_depth)))
+        self.max_depth = int(max_depth)     # the longest context tail a lookup can use
 
     def clear(self):
         _L().sv_suffix_clear(self._h)
@@ -202,7 +219,7 @@ class SuffixDrafter(_Handle):
             raise ValueError("sv_suffix_append rejected its arguments")
 
     def draft(self, problem_id: int, context, k: int = 16) -> np.ndarray:
-        c = _tok(context)
+        c = _tail(context, self.max_depth)
         out = np.empty(max(int(k), 1), np.int32)
         n = _L().sv_suffix_draft(self._h, int(problem_id), c.ctypes.data, c.size, int(k), out.ctypes.data)
         if n < 0:
@@ -211,10 +228,11 @@ class SuffixDrafter(_Handle):
 
     def draft_batch(self, problem_ids, contexts, k_max: int, max_lens=None, n_threads: int = 0):
         """Batched drafting, as NgramDrafter.draft_batch."""
-        return _draft_batch(_L().sv_suffix_draft_batch, self._h, problem_ids, contexts, k_max, max_lens, n_threads)
+        return _draft_batch(_L().sv_suffix_draft_batch, self._h, problem_ids, contexts, k_max, max_lens, n_threads,
+                            self.max_depth)
 
     def candidates(self, problem_id: int, context, f: int) -> np.ndarray:
-        c = _tok(context)
+        c = _tail(context, self.max_depth)
         out = np.empty(max(int(f), 1), np.int32)
         n = _L().sv_suffix_candidates(self._h, int(problem_id), c.ctypes.data, c.size, int(f), out.ctypes.data)
         if n < 0:
@@ -265,7 +283,10 @@ class FanoutPrefetcher:
     def prepare(self, key, prompt_id: int, context, draft) -> float:
         """Prefetch for request ``key`` (draft of at most k ids); returns the
         expected hit rate the allocation predicts."""
-        ctx, d = [int(x) for x in context], [int(x) for x in draft]
+        # a lookup reads at most the last max_n tokens of its context, and a
+        # branch only appends tokens to this one: its tail lies within ours
+        ctx = [int(x) for x in _tail(context, self.drafter.max_n)]
+        d = [int(x) for x in draft]
         if len(d) > self.k:
             raise ValueError(f"draft of {len(d)} ids, the prefetcher was built for k = {self.k}")
         f, coverage = self.budget.allocate(self.n_budget)
