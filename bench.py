@@ -377,6 +377,19 @@ def run_host(args):
                 break
         return n / (time.perf_counter() - t0)
     batch_1, batch_all = batch_rate(1), batch_rate(0)
+    # the same batches with their contexts already in one buffer
+    flat_batches = []
+    for pids, cs in batches:
+        off = np.zeros(len(cs) + 1, np.int64)
+        np.cumsum([len(c) for c in cs], out=off[1:])
+        flat_batches.append((pids, np.concatenate(cs).astype(np.int32), off))
+    n, t0 = 0, time.perf_counter()
+    for pids, flat, off in itertools.cycle(flat_batches):
+        ng.draft_batch_flat(pids, flat, off, 16, n_threads=1)
+        n += Bq
+        if time.perf_counter() - t0 > 3.0:
+            break
+    batch_flat = n / (time.perf_counter() - t0)
 
     # fan-out prefetch: the whole pipeline (budget, drafting ahead, serving
     # with a synchronous fallback) along fresh rollouts of the same prompts,
@@ -410,7 +423,7 @@ def run_host(args):
                                                     "10% token changes per rollout", "max_n": 6, "k": 16},
         "ngram_candidates_per_s": ng_cand, "suffix_draft_per_s": sx_rate, "prefetch_allocations_per_s": pf_rate,
         "ngram_batch_drafts_per_s": {"batch": Bq, "threads_1": batch_1, "threads_all": batch_all,
-                                     "hardware_threads": os.cpu_count()},
+                                     "flat_buffer_threads_1": batch_flat, "hardware_threads": os.cpu_count()},
         "fanout_prefetch": fanout,
         "table_build_s": build_s, "retained_tokens": ng.tokens, "mean_draft_len": float(np.mean(accepted)),
         "cpu_baseline": {"value": o_rate, "unit": "lookups/s", "cores": 1, "kind": "oracle",

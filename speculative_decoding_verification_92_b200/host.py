@@ -81,6 +81,33 @@ def _tail(a, n: int) -> np.ndarray:
     return _tok(a)[-n:]
 
 
+def _draft_batch_flat(fn, h, ids, flat, offsets, k_max, max_lens, n_threads):
+    """Batched drafting on contexts already laid out in one int32 buffer:
+    request b's context is flat[offsets[b]:offsets[b+1]].  No per-request
+    Python work, so the C++ lookups set the pace."""
+    ids = np.ascontiguousarray(np.asarray(ids, dtype=np.int64).reshape(-1))
+    B = ids.size
+    flat = np.ascontiguousarray(np.asarray(flat, dtype=np.int32).reshape(-1))
+    off = np.ascontiguousarray(np.asarray(offsets, dtype=np.int64).reshape(-1))
+    if off.size != B + 1:
+        raise ValueError(f"{B} ids need {B + 1} offsets, got {off.size}")
+    if B and (off[0] < 0 or np.any(np.diff(off) < 0) or off[-1] > flat.size):
+        raise ValueError("offsets must be non-decreasing and inside the buffer")
+    caps = None
+    if max_lens is not None:
+        caps = np.ascontiguousarray(np.asarray(max_lens, dtype=np.int32).reshape(-1))
+        if caps.size != B:
+            raise ValueError(f"{B} ids but {caps.size} max_lens")
+    tokens = np.empty((B, int(k_max)), np.int32)
+    lens = np.empty(B, np.int32)
+    rc = fn(h, B, ids.ctypes.data, flat.ctypes.data if flat.size else None, off.ctypes.data, int(k_max),
+            None if caps is None else caps.ctypes.data, int(n_threads),
+            tokens.ctypes.data if tokens.size else None, lens.ctypes.data)
+    if rc != 0:
+        raise ValueError("batched drafting rejected its arguments")
+    return tokens, lens
+
+
 def _draft_batch(fn, h, ids, contexts, k_max, max_lens, n_threads, tail):
     """Shared marshalling of the batched drafting calls: returns the
     drafted-id array [B, k_max] (-1 padded) and the lengths [B], both int32,
@@ -185,6 +212,12 @@ class NgramDrafter(_Handle):
         return _draft_batch(_L().sv_ngram_draft_batch, self._h, prompt_ids, contexts, k_max, max_lens, n_threads,
                             self.max_n)
 
+    def draft_batch_flat(self, prompt_ids, flat, offsets, k_max: int, max_lens=None, n_threads: int = 0):
+        """draft_batch on contexts laid out back to back in one int32 buffer
+        (request b: flat[offsets[b]:offsets[b+1]])."""
+        return _draft_batch_flat(_L().sv_ngram_draft_batch, self._h, prompt_ids, flat, offsets, k_max, max_lens,
+                                 n_threads)
+
     def candidates(self, prompt_id: int, context, f: int) -> np.ndarray:
         c = _tail(context, self.max_n)
         out = np.empty(max(int(f), 1), np.int32)
@@ -225,6 +258,12 @@ class SuffixDrafter(_Handle):
         if n < 0:
             raise ValueError("sv_suffix_draft rejected its arguments")
         return out[:n].copy()
+
+    def draft_batch_flat(self, problem_ids, flat, offsets, k_max: int, max_lens=None, n_threads: int = 0):
+        """Batched drafting on one flat context buffer, as
+        NgramDrafter.draft_batch_flat."""
+        return _draft_batch_flat(_L().sv_suffix_draft_batch, self._h, problem_ids, flat, offsets, k_max, max_lens,
+                                 n_threads)
 
     def draft_batch(self, problem_ids, contexts, k_max: int, max_lens=None, n_threads: int = 0):
         """Batched drafting, as NgramDrafter.draft_batch."""

@@ -378,6 +378,16 @@ def test_batched_drafting_matches_the_oracle_for_every_thread_count(which):
     # without caps every request may use k_max
     tok2, lens2 = c.draft_batch(ids, ctxs, k_max)
     assert np.all(lens2 >= lens)
+    # the same contexts laid out in one buffer
+    off = np.zeros(B + 1, np.int64)
+    np.cumsum([len(x) for x in ctxs], out=off[1:])
+    flat = np.concatenate([np.asarray(x, np.int32) for x in ctxs])
+    tok3, lens3 = c.draft_batch_flat(ids, flat, off, k_max, caps)
+    assert np.array_equal(tok3, tok) and np.array_equal(lens3, lens)
+    with pytest.raises(ValueError):
+        c.draft_batch_flat(ids, flat, off[:-1], k_max)                # one offset short
+    with pytest.raises(ValueError):
+        c.draft_batch_flat(ids, flat[:-1], off, k_max)                # offsets past the buffer
     # a batch large enough for several threads (at least 512 requests each)
     big = rng.integers(0, 8, size=2100)
     big_ctx = [ctxs[i % B] for i in range(big.size)]
