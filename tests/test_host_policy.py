@@ -702,3 +702,32 @@ def test_roofline_rejects_bad_arguments():
     assert math.isnan(host.spec_speedup(a, r, a, r, 4, 0, 0.5, 10))
     assert math.isnan(host.spec_speedup(a, r, a, r, 4, 5, 1.5, 10))
     assert math.isnan(host.roofline_time(a, host.Roofline(0.0, 1.0, 0.0), 1, 1, 1))
+
+
+# ---------------------------------------------------------------------------
+# planted slips in the host oracle (on the CPU): each must fail a pin
+
+def _work_without_attention(a, B, q, n):
+    return 2.0 * a["params"] * B * q, a["params"] * a["weight_bytes"] + 2.0 * a["layers"] * a["kv_heads"] * \
+        a["head_dim"] * a["kv_bytes"] * B * n
+
+
+def _work_k_only(a, B, q, n):
+    flops = 2.0 * a["params"] * B * q + 4.0 * a["layers"] * a["width"] * B * q * n
+    return flops, a["params"] * a["weight_bytes"] + a["layers"] * a["kv_heads"] * a["head_dim"] * a["kv_bytes"] * B * n
+
+
+def _cycle_without_bonus(alpha, k):
+    return sum(alpha ** i for i in range(k))
+
+
+@pytest.mark.parametrize("name,slip,pin", [
+    ("attention flops dropped", ("roofline_work", _work_without_attention), test_pin_roofline_work_against_explicit_tensors),
+    ("V cache not counted", ("roofline_work", _work_k_only), test_pin_roofline_work_against_explicit_tensors),
+    ("no token drawn after the accepted prefix", ("accepted_per_cycle", _cycle_without_bonus),
+     test_pin_speedup_special_cases),
+])
+def test_host_oracle_slips_fail_a_pin(monkeypatch, name, slip, pin):
+    monkeypatch.setattr(ho, slip[0], slip[1])
+    with pytest.raises(AssertionError):
+        pin()
