@@ -731,3 +731,45 @@ def test_host_oracle_slips_fail_a_pin(monkeypatch, name, slip, pin):
     monkeypatch.setattr(ho, slip[0], slip[1])
     with pytest.raises(AssertionError):
         pin()
+
+
+def _draft_from_oldest(self, pid, ctx, k=16):
+    n, occ = self._longest(pid, ctx)
+    if n == 0 or k == 0:
+        return []
+    r, p = occ[-1]                       # the oldest occurrence instead of the newest
+    return r[p:p + k]
+
+
+def _begin_step_keeping_everything(self):
+    self.step += 1                       # no eviction: the window is ignored
+
+
+def _longest_uncapped(self, pid, ctx):
+    ctx = [int(x) for x in ctx]
+    for n in range(len(ctx), 0, -1):     # n not capped at max_n
+        occ = list(self._occurrences(pid, ctx[-n:]))
+        if occ:
+            return n, occ
+    return 0, []
+
+
+def _trajectory_patience_one(lengths, taus, up=0.7, down=0.4, patience=2):
+    return _ORIGINAL_TRAJECTORY(lengths, taus, up, down, 1)
+
+
+_ORIGINAL_TRAJECTORY = ho.draft_length_trajectory
+
+
+@pytest.mark.parametrize("name,target,attr,slip,pin", [
+    ("oldest occurrence", ho.NgramOracle, "draft", _draft_from_oldest, test_pin_ngram_window_and_recency),
+    ("window ignored", ho.NgramOracle, "begin_step", _begin_step_keeping_everything,
+     test_pin_ngram_window_and_recency),
+    ("n not capped", ho.NgramOracle, "_longest", _longest_uncapped, test_pin_ngram_longest_match_capped_at_n),
+    ("one-step patience", ho, "draft_length_trajectory", _trajectory_patience_one,
+     test_pin_draft_length_rises_5_7_9_11_as_acceptance_grows),
+])
+def test_host_policy_slips_fail_a_pin(monkeypatch, name, target, attr, slip, pin):
+    monkeypatch.setattr(target, attr, slip)
+    with pytest.raises(AssertionError):
+        pin()
