@@ -773,3 +773,49 @@ def test_host_policy_slips_fail_a_pin(monkeypatch, name, target, attr, slip, pin
     monkeypatch.setattr(target, attr, slip)
     with pytest.raises(AssertionError):
         pin()
+
+
+def _draft_first_seen(self, pid, ctx, k=16):
+    ctx = [int(x) for x in ctx]
+    out = []
+    while len(out) < k:
+        cnt = self._longest(pid, ctx)
+        if not cnt:
+            break
+        t = next(iter(cnt))              # the first follower seen, not the most frequent
+        out.append(t)
+        ctx.append(t)
+    return out
+
+
+_ORIGINAL_ESTIMATES = ho.prefetch_estimates
+
+
+def _estimates_whole_history(obs, k, fmax, window):
+    return _ORIGINAL_ESTIMATES(obs, k, fmax, len(obs))     # the window ignored
+
+
+def _allocate_by_branch_share(obs, k, fmax, window, budget):
+    n, P, cov = ho.prefetch_estimates(obs, k, fmax, window)
+    f = [0] * (k + 1)
+    if n == 0:
+        return f, 0.0
+    for _ in range(budget):                                 # the likeliest open branch, whatever it gains
+        j = max((j for j in range(k + 1) if f[j] < fmax), key=lambda j: P[j], default=None)
+        if j is None:
+            break
+        f[j] += 1
+    return f, ho.expected_coverage(P, cov, f)
+
+
+@pytest.mark.parametrize("name,target,attr,slip,pin", [
+    ("first follower, not the most frequent", ho.SuffixOracle, "draft", _draft_first_seen,
+     test_pin_suffix_frequency_and_immediate_insertion),
+    ("window ignored", ho, "prefetch_estimates", _estimates_whole_history, test_pin_prefetch_window_is_causal),
+    ("budget by branch share alone", ho, "prefetch_allocate", _allocate_by_branch_share,
+     test_pin_prefetch_all_accepted_branch_needs_one_candidate),
+])
+def test_more_host_policy_slips_fail_a_pin(monkeypatch, name, target, attr, slip, pin):
+    monkeypatch.setattr(target, attr, slip)
+    with pytest.raises(AssertionError):
+        pin()
