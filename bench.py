@@ -23,6 +23,11 @@ Rank 0 prints one JSON line.
 With N > 1 (torchrun), every rank verifies its own batch (weak scaling); no
 collective touches the data path, only the timing barrier and the max over
 ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+
+``--host`` times the host-side components instead, on one CPU core and a
+synthetic rollout history: per-request and batched n-gram drafting (lists
+and one flat buffer), ranked candidates, suffix drafting, the prefetch
+budget, and the fan-out prefetch pipeline's hit rate against its prediction.
 """
 from __future__ import annotations
 
