@@ -39,7 +39,7 @@
  *            at the first rejection instead of at the first position; the
  *            ablation's hard cut-off gives zero weight after it.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *  - residual = normalise(max(0, p - q)) (the plain reading of "target minus what
  *    the draft proposed");
  *  - all drafts accepted -> bonus token drawn from the target row L (row k+1);
