@@ -40,8 +40,8 @@
  *            ablation's hard cut-off gives zero weight after it.
  *
  * Readings where the pages are silent:
- *  - residual = normalise(max(0, p - q)) (the plain reading of "target minus what
- *    the draft proposed");
+ *  - residual = normalise(max(0, p - q)), the plain reading of a redraw from
+ *    the target with the draft's share taken out;
  *  - all drafts accepted -> bonus token drawn from the target row L (row k+1);
  *  - target and draft logits are both divided by the same temperature T;
  *  - uniforms[b*(k_max+1) + i] is the acceptance draw for draft i; the separate

@@ -19,8 +19,10 @@ from oracle import host_policy as ho
 # section "📓 NgramRL：每道题配一本活页草稿本")
 
 def test_pin_ngram_page_example():
-    """A generation ending in "so the final answer is" is drafted with the
-    continuation the prompt's earlier rollout wrote after that prefix."""
+    """The page's worked example, with token ids standing for its words: a
+    generation whose tail is the phrase before a final answer is drafted
+    with the continuation an earlier rollout of the same prompt wrote after
+    that phrase (the answer, a comma, and the reasoning that follows)."""
     SO, FINAL, ANSWER, IS, N42, COMMA, BECAUSE = 101, 102, 103, 104, 42, 7, 105
     tail = [N42, COMMA, BECAUSE] + list(range(200, 220))
     rollout = [1, 2, 3, SO, FINAL, ANSWER, IS] + tail
