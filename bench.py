@@ -3,11 +3,12 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
-One step = one ``spec_verify`` call over one batch of the synthetic
-quantized-self-draft workload (B=64 requests, k=8 drafts, V=151,936, bf16
-logits, T=1) with its inputs already resident in HBM: the row-statistics
-kernel over every used row, then the acceptance scan and the final draw.
-Rank 0 prints one JSON line.
+One step = one ``spec_verify`` call over one batch of a synthetic workload
+with its inputs already resident in HBM: the row-statistics kernel over every
+used row, then the acceptance scan and the final draw.  The default workload
+is the largest single-GPU one, the length-aware-budgets batch (B=256,
+k_max=12, per-request draft lengths in {0, 4, 12}, V=128,256, fp32 logits,
+T=1, about 1 GB of logits read per step).  Rank 0 prints one JSON line.
 
 * value        verified draft positions/s over all ranks (sum of draft
                lengths per call x calls / max-over-ranks device time)
@@ -15,10 +16,14 @@ Rank 0 prints one JSON line.
                (spec_verify_host): pinned host inputs copied in, results
                copied out, every step
 * roofline     the row-statistics kernel: algorithmic bytes (every logit of
-               every used row, read once) / its CUDA-event time, against the
-               measured HBM copy bandwidth
-* cpu_baseline the CPU oracle on the host cores (single thread), on a bounded
-               sample of the same workload
+               every used row, read once) / its mean CUDA-event time over a
+               separate pass of at least 10 launches, against the measured
+               HBM copy bandwidth; the whole step's bandwidth beside it
+* per_config   the same figures for the four other workloads (1 GPU), each
+               with a parity spot check (outputs well formed, host entry
+               point equal to the device entry point)
+* cpu_baseline the CPU oracle on every hardware thread of the host (and
+               single-threaded on a sample), on the same workload
 
 With N > 1 (torchrun), every rank verifies its own batch (weak scaling); no
 collective touches the data path, only the timing barrier and the max over
@@ -73,15 +78,18 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=2, choices=sorted(CONFIGS))
+    ap.add_argument("--config", type=int, default=5, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--stats-kernel", default="auto", choices=["auto", "tma", "vec16", "scalar"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--greedy", action="store_true", help="time the greedy (prefix-match) form instead")
-    ap.add_argument("--event-every", type=int, default=16,
-                    help="bracket the row-statistics kernel with events on every N-th timed step")
+    ap.add_argument("--k1-samples", type=int, default=50,
+                    help="launches of the row-statistics kernel timed with events (at least 10)")
+    ap.add_argument("--per-config-steps", type=int, default=200,
+                    help="timed steps of each other workload in the per_config block")
+    ap.add_argument("--no-per-config", action="store_true", help="time the chosen workload only")
     ap.add_argument("--host", action="store_true",
                     help="time the host-side drafters and prefetch budget instead (CPU only)")
     return ap.parse_args()
@@ -242,68 +250,105 @@ class ClockSampler:
 # CPU oracle timing
 
 
-def time_oracle(w, n_requests: int, seconds: float, greedy=False, min_reps=1):
-    """Run the oracle on the first n_requests of the batch until `seconds`
-    have passed (at least min_reps times); returns (positions/s, reps,
-    positions per rep, seconds)."""
+def _request_slices(w, n_parts: int):
+    """Contiguous request ranges of about equal row counts (the oracle's work
+    is proportional to the rows it reads)."""
+    rows = (w.draft_lens.astype(np.int64) + 1) * (2 if w.draft is not None else 1)
+    cum = np.concatenate([[0], np.cumsum(rows)])
+    cuts = [int(np.searchsorted(cum, cum[-1] * i / n_parts)) for i in range(n_parts + 1)]
+    cuts[0], cuts[-1] = 0, w.B
+    return [slice(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+
+
+def _oracle_call(orc, w, sl, greedy):
+    lens = None if w.lens is None else w.lens[sl]
+    orc.verify(w.target[sl], None if (greedy or w.draft is None) else w.draft[sl], w.tokens[sl], lens,
+               None if greedy else w.uniforms[sl].astype(np.float64), w.temperature, greedy, V=w.V)
+
+
+def time_oracle(w, seconds: float, greedy=False, threads: int = 1, n_requests: int | None = None):
+    """Run the oracle over the first n_requests (default all) of the batch,
+    split into `threads` contiguous request ranges verified concurrently (the
+    oracle's C entry point releases the GIL; each request is still verified
+    sequentially), until `seconds` have passed.  Returns (positions/s, passes,
+    positions per pass, seconds, threads used)."""
+    from concurrent.futures import ThreadPoolExecutor
     from oracle import default
     orc = default()
-    sl = slice(0, n_requests)
-    lens = None if w.lens is None else w.lens[sl]
-    u = w.uniforms[sl].astype(np.float64)
-    positions = int(w.draft_lens[sl].sum())
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        orc.verify(w.target[sl], None if (greedy or w.draft is None) else w.draft[sl], w.tokens[sl], lens,
-                   None if greedy else u, w.temperature, greedy, V=w.V)
-        reps += 1
-        el = time.perf_counter() - t0
-        if reps >= min_reps and el >= seconds:
-            break
-    return positions * reps / el, reps, positions, el
+    n = w.B if n_requests is None else max(1, min(w.B, n_requests))
+    sub = w if n == w.B else _sub_workload(w, n)
+    slices = _request_slices(sub, max(1, threads))
+    positions = int(sub.draft_lens.sum())
+    passes, t0 = 0, time.perf_counter()
+    with ThreadPoolExecutor(max_workers=len(slices)) as ex:
+        while True:
+            list(ex.map(lambda sl: _oracle_call(orc, sub, sl, greedy), slices))
+            passes += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    return positions * passes / el, passes, positions, el, len(slices)
+
+
+def _sub_workload(w, n):
+    """The first n requests of a workload (views, no copies)."""
+    import dataclasses
+    return dataclasses.replace(w, B=n, target=w.target[:n], draft=None if w.draft is None else w.draft[:n],
+                               tokens=w.tokens[:n], lens=None if w.lens is None else w.lens[:n],
+                               uniforms=w.uniforms[:n], favoured=None if w.favoured is None else w.favoured[:n])
+
+
+def oracle_baseline(w, seconds: float, greedy=False):
+    """The oracle on the host's cores: single-threaded on a sample of the
+    batch, then on the whole batch with one thread per hardware thread."""
+    cores = os.cpu_count() or 1
+    per_req = stats_pass_bytes(w, greedy) / max(1, w.B)
+    n1 = int(max(1, min(w.B, 2e9 / max(per_req, 1))))        # ~1-2 s of single-threaded work per pass
+    v1, p1, pos1, el1, _ = time_oracle(w, seconds / 2, greedy, threads=1, n_requests=n1)
+    vn, pn, posn, eln, used = time_oracle(w, seconds / 2, greedy, threads=cores)
+    return {"value": vn, "unit": UNIT, "cores": used, "host_cores": cores, "kind": "oracle",
+            "single_thread_value": v1,
+            "sample": f"all {w.B} requests ({posn} draft positions) x {pn} passes in {eln:.1f} s on {used} threads "
+                      f"(contiguous request ranges, one per hardware thread); single thread: first {n1} requests "
+                      f"({pos1} positions) x {p1} passes in {el1:.1f} s; plain C, fp64"}
 
 
 # ---------------------------------------------------------------------------
 
 
 def run_reference(args):
-    """CPU oracle arm: rank 0 alone; every step verifies a bounded sample."""
+    """CPU oracle arm: rank 0 alone, on every hardware thread of the host;
+    every step verifies a bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     w = make_rank_workload(args.config, 0)
-    from oracle import default
-    orc = default()
+    cores = os.cpu_count() or 1
     # calibrate the per-request cost, then size the per-step sample so that
     # warm-up + steps stay within about two minutes
     t0 = time.perf_counter()
-    orc.verify(w.target[:1], None if w.draft is None else w.draft[:1], w.tokens[:1],
-               None if w.lens is None else w.lens[:1], w.uniforms[:1].astype(np.float64), w.temperature,
-               args.greedy, V=w.V)
+    _oracle_call(__import__("oracle").default(), w, slice(0, 1), args.greedy)
     per_req = max(time.perf_counter() - t0, 1e-4)
     budget = 120.0 / max(1, args.steps + args.warmup)
-    n_req = int(max(1, min(w.B, budget // per_req)))
-    sl = slice(0, n_req)
-    lens = None if w.lens is None else w.lens[sl]
-    u = w.uniforms[sl].astype(np.float64)
-    draft = None if (w.draft is None or args.greedy) else w.draft[sl]
-    positions = int(w.draft_lens[sl].sum())
+    n_req = int(max(1, min(w.B, cores * budget // per_req)))
+    sub = w if n_req == w.B else _sub_workload(w, n_req)
     for _ in range(args.warmup):
-        orc.verify(w.target[sl], draft, w.tokens[sl], lens, u, w.temperature, args.greedy, V=w.V)
-    times = []
+        time_oracle(sub, 0.0, args.greedy, threads=cores)
+    times, positions, used = [], int(sub.draft_lens.sum()), 1
     for _ in range(args.steps):
-        t0 = time.perf_counter()
-        orc.verify(w.target[sl], draft, w.tokens[sl], lens, u, w.temperature, args.greedy, V=w.V)
-        times.append(time.perf_counter() - t0)
+        v, passes, positions, el, used = time_oracle(sub, 0.0, args.greedy, threads=cores)
+        times.append(el / passes)
     total = sum(times)
     value = positions * args.steps / total
-    sample = f"first {n_req} of {w.B} requests ({positions} draft positions) per step"
+    sample = (f"first {n_req} of {w.B} requests ({positions} draft positions) per step, "
+              f"on {used} threads (one contiguous request range each)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_desc(w, args.config),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "host_cores": cores, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -447,6 +492,182 @@ def main():
     return run_ours_impl(args)
 
 
+class DeviceWorkload:
+    """One workload resident on the device, with its output buffers and
+    workspace, and the call that verifies it."""
+
+    def __init__(self, sv, torch, dev, stream, w, greedy, kernel):
+        self.sv, self.torch, self.dev, self.stream, self.w = sv, torch, dev, stream, w
+        self.greedy, self.kernel = greedy, kernel
+        self.is_bf16 = w.dtype == "bf16"
+        t = lambda a, bf=False: (torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16) if bf
+                                 else torch.from_numpy(np.ascontiguousarray(a))).to(dev)
+        self.target = t(w.target, self.is_bf16)
+        self.draft = None if (w.draft is None or greedy) else t(w.draft, self.is_bf16)
+        self.tokens = t(w.tokens)
+        self.lens = None if w.lens is None else t(w.lens)
+        self.uniforms = None if greedy else t(w.uniforms)
+        self.out = (torch.empty(w.B, dtype=torch.int32, device=dev),
+                    torch.empty(w.B, w.k_max + 1, dtype=torch.int32, device=dev))
+        self.ws = torch.empty(max(sv.workspace_bytes(w.B, w.k_max, w.V, sv.BF16 if self.is_bf16 else sv.F32), 256),
+                              dtype=torch.uint8, device=dev)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.in_bytes = input_bytes(w, greedy)
+        self.flush_buf = None
+        if self.in_bytes < 2 * l2:
+            self.flush_buf = torch.empty(4 * l2 // 4, dtype=torch.int32, device=dev)
+        self.l2_note = (f"inputs {self.in_bytes / 1e6:.1f} MB > 2 x L2 ({l2 / 2**20:.0f} MiB): no flush"
+                        if self.flush_buf is None else
+                        f"inputs {self.in_bytes / 1e6:.1f} MB < 2 x L2: L2 flushed (write "
+                        f"{self.flush_buf.numel() * 4 / 2**20:.0f} MiB) before every step, outside each step's events")
+
+    def step(self, events=None):
+        w = self.w
+        self.sv.spec_verify(self.target, self.draft, self.tokens, self.lens, self.uniforms, w.temperature,
+                            self.greedy, V=w.V, out=self.out, workspace=self.ws, stream=self.stream,
+                            stats_kernel=self.kernel, events=events)
+
+    def event(self):
+        e = self.torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        return e
+
+    def time_steps(self, steps, warmup, barrier=lambda: None):
+        """Time `steps` calls; returns (device ms over the timed calls,
+        region ms).  Without an L2 flush the calls run back to back between
+        two events; with one, every call is bracketed by its own events and
+        the flush stays outside them."""
+        torch = self.torch
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        step_ev = [(None, None)] * steps
+        g0 = g1 = None
+        barrier()
+        torch.cuda.synchronize()
+        if self.flush_buf is None:
+            g0 = self.event()
+            for _ in range(steps):
+                self.step()
+            g1 = self.event()
+        else:
+            step_ev = []
+            for i in range(steps):
+                self.flush_buf.fill_(i)
+                a = self.event()
+                self.step()
+                step_ev.append((a, self.event()))
+        torch.cuda.synchronize()
+        barrier()
+        if self.flush_buf is None:
+            region = g0.elapsed_time(g1)
+            return region, region
+        per = [a.elapsed_time(b) for a, b in step_ev]
+        return sum(per), sum(per)
+
+    def time_k1(self, samples):
+        """The row-statistics kernel alone: `samples` calls, each with events
+        recorded just before and after that kernel on the launching stream
+        (a separate pass, so the events do not disturb the timed steps).
+        Returns the per-launch times in ms."""
+        torch = self.torch
+        ev = []
+        for i in range(samples):
+            if self.flush_buf is not None:
+                self.flush_buf.fill_(i)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            self.step(events=(a, b))
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    def host_check(self):
+        """Parity spot check of the device outputs: every accept length lies
+        in [0, L_b], the accepted prefix repeats the drafts, the emitted
+        token is a vocabulary id and -1 fills the rest; and the host entry
+        point (spec_verify_host, host buffers) returns the same outputs."""
+        torch, w = self.torch, self.w
+        self.step()
+        torch.cuda.synchronize()
+        g_len = self.out[0].cpu().numpy()
+        g_tok = self.out[1].cpu().numpy()
+        L = w.draft_lens
+        ok = bool(np.all((g_len >= 0) & (g_len <= L)))
+        for b in range(w.B) if ok else ():
+            j = int(g_len[b])
+            ok &= bool(np.array_equal(g_tok[b, :j], w.tokens[b, :j]) and 0 <= g_tok[b, j] < w.V
+                       and np.all(g_tok[b, j + 1:] == -1))
+        h = self.host_buffers()
+        self.sv.spec_verify_host(*h["inputs"], w.temperature, self.greedy, V=w.V, out=h["out"],
+                                 staging=h["staging"], workspace=self.ws, stream=self.stream)
+        torch.cuda.synchronize()
+        same = bool(np.array_equal(h["out"][0].numpy(), g_len) and np.array_equal(h["out"][1].numpy(), g_tok))
+        return g_len, {"outputs_valid": ok, "host_entry_point_matches": same}
+
+    def host_buffers(self):
+        if getattr(self, "_host", None) is None:
+            torch, w = self.torch, self.w
+            pin = lambda a, bf=False: (torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16) if bf
+                                       else torch.from_numpy(np.ascontiguousarray(a))).pin_memory()
+            h_draft = None if self.draft is None else pin(w.draft, self.is_bf16)
+            h_lens = None if w.lens is None else pin(w.lens)
+            inputs = (pin(w.target, self.is_bf16), h_draft, pin(w.tokens), h_lens,
+                      None if self.greedy else pin(w.uniforms))
+            out = (torch.empty(w.B, dtype=torch.int32).pin_memory(),
+                   torch.empty(w.B, w.k_max + 1, dtype=torch.int32).pin_memory())
+            n = self.sv.host_staging_bytes(w.B, w.k_max, w.V, self.sv.BF16 if self.is_bf16 else self.sv.F32,
+                                           has_draft=h_draft is not None, has_lens=h_lens is not None)
+            self._host = {"inputs": inputs, "out": out,
+                          "staging": torch.empty(max(n, 256), dtype=torch.uint8, device=self.dev)}
+        return self._host
+
+    def release(self):
+        for name in ("target", "draft", "tokens", "lens", "uniforms", "out", "ws", "flush_buf", "_host"):
+            setattr(self, name, None)
+
+
+def reread_bytes(w, g_len, greedy=False) -> int:
+    """Algorithmic bytes of the final draw: the target row j again, plus the
+    draft row j when a draft with logits was rejected there (greedy: none)."""
+    if greedy:
+        return 0
+    L = w.draft_lens
+    resid = (g_len < L) & (w.draft is not None)
+    return int((1 + resid.astype(np.int64)).sum()) * w.V * w.esize
+
+
+def launches_per_call(B: int, greedy: bool) -> int:
+    """Kernels one spec_verify call launches: the row-statistics kernel per
+    block of up to 4096 requests, then the scan-and-draw kernel per block of
+    up to 65535 requests."""
+    return math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + math.ceil(B / MAX_REQUESTS_PER_DRAW_LAUNCH)
+
+
+def config_record(dw, cfg, steps, warmup, k1_samples, peak):
+    """Per-workload figures for the per_config block of the bench line."""
+    w = dw.w
+    dev_ms, _ = dw.time_steps(steps, warmup)
+    k1 = dw.time_k1(k1_samples)
+    g_len, parity = dw.host_check()
+    alg = stats_pass_bytes(w, dw.greedy)
+    rr = reread_bytes(w, g_len, dw.greedy)
+    step_ms = dev_ms / steps
+    k1_med, k1_mean = float(np.median(k1)), statistics.fmean(k1)
+    return {
+        "workload": workload_desc(w, cfg)["workload"], "l2": dw.l2_note, "steps": steps,
+        "positions_per_s": w.positions * steps / (dev_ms / 1e3),
+        "step_us": 1e3 * step_ms, "step_gbs": alg / (step_ms / 1e3) / 1e9,
+        "step_frac": alg / (step_ms / 1e3) / 1e9 / peak,
+        "step_gbs_with_reread": (alg + rr) / (step_ms / 1e3) / 1e9,
+        "stats_bytes": alg, "reread_bytes": rr,
+        "k1_samples": len(k1), "k1_us_median": 1e3 * k1_med, "k1_us_mean": 1e3 * k1_mean,
+        "k1_gbs_median": alg / (k1_med / 1e3) / 1e9, "k1_frac_median": alg / (k1_med / 1e3) / 1e9 / peak,
+        "k1_frac_mean": alg / (k1_mean / 1e3) / 1e9 / peak,
+        "accept_rate": float(g_len.sum() / max(1, w.positions)), "mean_accept_len": float(g_len.mean()),
+        "parity": parity,
+    }
+
+
 def run_ours_impl(args):
     import torch
     import torch.distributed as dist
@@ -469,130 +690,62 @@ def run_ours_impl(args):
             dist.barrier()
 
     sv.library()  # build / load before timing anything
-    w = make_rank_workload(args.config, rank)
     greedy = bool(args.greedy)
     kernel = {"auto": sv.StatsKernel.AUTO, "tma": sv.StatsKernel.TMA, "vec16": sv.StatsKernel.VEC16,
               "scalar": sv.StatsKernel.SCALAR}[args.stats_kernel]
-
-    def dev_tensor(a, bf16=False):
-        t = torch.from_numpy(np.ascontiguousarray(a))
-        if bf16:
-            t = t.view(torch.bfloat16)
-        return t.to(dev)
-
-    is_bf16 = w.dtype == "bf16"
-    target = dev_tensor(w.target, is_bf16)
-    draft = None if (w.draft is None or greedy) else dev_tensor(w.draft, is_bf16)
-    tokens = dev_tensor(w.tokens)
-    lens = None if w.lens is None else dev_tensor(w.lens)
-    uniforms = None if greedy else dev_tensor(w.uniforms)
-    out = (torch.empty(w.B, dtype=torch.int32, device=dev),
-           torch.empty(w.B, w.k_max + 1, dtype=torch.int32, device=dev))
-    ws = torch.empty(max(sv.workspace_bytes(w.B, w.k_max, w.V, sv.BF16 if is_bf16 else sv.F32), 256),
-                     dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    in_bytes = input_bytes(w, greedy)
-    flush_buf = None
-    if in_bytes < 2 * l2:
-        flush_buf = torch.empty(4 * l2 // 4, dtype=torch.int32, device=dev)
-    l2_note = (f"inputs {in_bytes / 1e6:.1f} MB > 2 x L2 ({l2 / 2**20:.0f} MiB): no flush" if flush_buf is None
-               else f"inputs {in_bytes / 1e6:.1f} MB < 2 x L2: L2 flushed (write {flush_buf.numel() * 4 / 2**20:.0f}"
-                    f" MiB) before every step, outside each step's events")
-
-    def step(events=None):
-        sv.spec_verify(target, draft, tokens, lens, uniforms, w.temperature, greedy, V=w.V, out=out,
-                       workspace=ws, stream=stream, stats_kernel=kernel, events=events)
-
-    def new_event():
-        e = torch.cuda.Event(enable_timing=True)
-        e.record(stream)
-        return e
+    peak, peak_kind = measured_peak()
+    w = make_rank_workload(args.config, rank)
+    dw = DeviceWorkload(sv, torch, dev, stream, w, greedy, kernel)
 
     K, W = args.steps, args.warmup
-    for _ in range(W):
-        step()
-    torch.cuda.synchronize()
-    # Events cost a few microseconds each on the stream, so only every
-    # EVENT_EVERY-th step brackets the row-statistics kernel; steps are timed
-    # individually only when the L2 is flushed between them.
-    every = max(1, args.event_every)
-    k1_ev = {i: (new_event(), new_event()) for i in range(0, K, every)}
-    step_ev = [(new_event(), new_event()) for _ in range(K)] if flush_buf is not None else None
-    g0, g1 = new_event(), new_event()
-    torch.cuda.synchronize()
-
-    barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
-        g0.record(stream)
-        for i in range(K):
-            if flush_buf is not None:
-                flush_buf.fill_(i)
-                step_ev[i][0].record(stream)
-            step(events=k1_ev.get(i))
-            if flush_buf is not None:
-                step_ev[i][1].record(stream)
-        g1.record(stream)
-        torch.cuda.synchronize()
-    barrier()
-
-    k1_ms = [a.elapsed_time(b) for a, b in k1_ev.values()]
-    region_ms = g0.elapsed_time(g1)
-    step_ms = [a.elapsed_time(b) for a, b in step_ev] if step_ev is not None else [region_ms / K]
-    t_rank = sum(step_ms) if flush_buf is not None else region_ms
+        t_rank, region_ms = dw.time_steps(K, W, barrier)
     t_max = max_over_ranks(t_rank, dev)
     positions = w.positions
     value = aggregate_value(n, positions, K, t_max)
     ms_per_step = t_max / K
 
-    # parity spot check of the timed outputs (host side, cheap): accept lengths in range
-    g_len = out[0].cpu().numpy()
-    assert np.all((g_len >= 0) & (g_len <= w.draft_lens)), "timed run produced invalid outputs"
+    # the row-statistics kernel alone, in its own pass of at least 10 launches
+    k1_ms = dw.time_k1(max(args.k1_samples, 10))
+    g_len, parity = dw.host_check()
+    assert parity["outputs_valid"], "timed run produced invalid outputs"
+    assert parity["host_entry_point_matches"], "host entry point disagrees with device entry point"
     accept_rate = float(g_len.sum() / max(1, positions))
 
     # ---------------- end to end through the host entry point ----------------
     e2e = None
     if args.e2e_steps > 0:
-        pin = lambda a, bf=False: (torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16) if bf
-                                   else torch.from_numpy(np.ascontiguousarray(a))).pin_memory()
-        h_target = pin(w.target, is_bf16)
-        h_draft = None if draft is None else pin(w.draft, is_bf16)
-        h_tokens, h_lens = pin(w.tokens), (None if w.lens is None else pin(w.lens))
-        h_u = None if greedy else pin(w.uniforms)
-        h_out = (torch.empty(w.B, dtype=torch.int32).pin_memory(),
-                 torch.empty(w.B, w.k_max + 1, dtype=torch.int32).pin_memory())
-        staging = torch.empty(sv.host_staging_bytes(w.B, w.k_max, w.V, sv.BF16 if is_bf16 else sv.F32,
-                                                    has_draft=h_draft is not None, has_lens=h_lens is not None),
-                              dtype=torch.uint8, device=dev)
+        h = dw.host_buffers()
 
         def e2e_step():
-            sv.spec_verify_host(h_target, h_draft, h_tokens, h_lens, h_u, w.temperature, greedy, V=w.V,
-                                out=h_out, staging=staging, workspace=ws, stream=stream)
+            sv.spec_verify_host(*h["inputs"], w.temperature, greedy, V=w.V, out=h["out"], staging=h["staging"],
+                                workspace=dw.ws, stream=stream)
 
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize()
-        ev = [(new_event(), new_event()) for _ in range(args.e2e_steps)]
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.e2e_steps)]
         barrier()
         torch.cuda.synchronize()
-        for i in range(args.e2e_steps):
-            ev[i][0].record(stream)
+        for a, b in ev:
+            a.record(stream)
             e2e_step()
-            ev[i][1].record(stream)
+            b.record(stream)
         torch.cuda.synchronize()
         barrier()
         e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
-        assert np.array_equal(h_out[0].numpy(), g_len), "host entry point disagrees with device entry point"
+        assert np.array_equal(h["out"][0].numpy(), g_len), "host entry point disagrees with device entry point"
         e2e = {"value": aggregate_value(n, positions, args.e2e_steps, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": int(h_out[0].nbytes + h_out[1].nbytes),
+               "h2d_bytes_per_step": dw.in_bytes,
+               "d2h_bytes_per_step": int(h["out"][0].nbytes + h["out"][1].nbytes),
                "steps": args.e2e_steps, "ms_per_step": e2e_ms / args.e2e_steps}
 
     # ---------------- roofline of the row-statistics kernel ----------------
-    peak, peak_kind = measured_peak()
     alg = stats_pass_bytes(w, greedy)
-    k1_mean = statistics.fmean(k1_ms)
+    rr = reread_bytes(w, g_len, greedy)
+    k1_mean, k1_med = statistics.fmean(k1_ms), float(np.median(k1_ms))
     achieved = alg / (k1_mean / 1e3) / 1e9
     variant = "tma" if args.stats_kernel == "auto" else args.stats_kernel
     traffic = committed_traffic(variant, args.config)
@@ -600,34 +753,54 @@ def run_ours_impl(args):
                 "traffic": traffic, "peak_kind": f"{peak_kind} (copy bandwidth, MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s",
                 "kernel": f"row_stats ({variant})", "algorithmic_bytes_per_launch": alg,
-                "kernel_ms": k1_mean, "kernel_ms_p10": float(np.percentile(k1_ms, 10)),
-                "whole_step_gbs": alg / (ms_per_step / 1e3) / 1e9}
+                "kernel_ms": k1_mean, "kernel_ms_median": k1_med,
+                "kernel_ms_p10": float(np.percentile(k1_ms, 10)), "kernel_samples": len(k1_ms),
+                "frac_median": alg / (k1_med / 1e3) / 1e9 / peak,
+                "whole_step_gbs": alg / (ms_per_step / 1e3) / 1e9,
+                "whole_step_frac": alg / (ms_per_step / 1e3) / 1e9 / peak,
+                "reread_bytes_per_step": rr,
+                "whole_step_gbs_with_reread": (alg + rr) / (ms_per_step / 1e3) / 1e9}
 
-    launches_per_call = math.ceil(w.B / MAX_REQUESTS_PER_STATS_LAUNCH) + math.ceil(w.B / MAX_REQUESTS_PER_DRAW_LAUNCH)
+    cfgd = workload_desc(w, args.config)
+    cfgd.update({"parallelism": f"replicas{n}" if n > 1 else "single",
+                 "sharding": "each rank verifies its own batch; no data-path collective",
+                 "l2": dw.l2_note, "stats_kernel": variant, "greedy": greedy})
+    dw.release()
+
+    # ---------------- the other workloads (rank 0, N = 1) ----------------
+    per_config = None
+    if rank == 0 and n == 1 and not args.no_per_config:
+        per_config = {}
+        for cfg in sorted(CONFIGS):
+            if cfg == args.config:
+                continue
+            wc = make_rank_workload(cfg, 0)
+            dc = DeviceWorkload(sv, torch, dev, stream, wc, greedy, kernel)
+            per_config[str(cfg)] = config_record(dc, cfg, args.per_config_steps, max(W, 3),
+                                                 max(args.k1_samples, 10), peak)
+            dc.release()
+            del dc
+            torch.cuda.empty_cache()
 
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
     cpu = None
     if rank == 0 and n == 1 and not args.no_cpu_baseline:
-        v, reps, pos, el = time_oracle(w, w.B, args.cpu_seconds, greedy)
-        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"whole batch ({w.B} requests, {pos} draft positions) x {reps} passes, {el:.1f} s,"
-                         f" single-threaded C, fp64"}
+        cpu = oracle_baseline(w, args.cpu_seconds, greedy)
 
     if rank == 0:
-        cfgd = workload_desc(w, args.config)
-        cfgd.update({"parallelism": f"replicas{n}" if n > 1 else "single",
-                     "sharding": "each rank verifies its own batch; no data-path collective",
-                     "l2": l2_note, "stats_kernel": variant, "greedy": greedy})
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": K, "warmup": W,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic", "config": cfgd,
-            "e2e": e2e, "gpu_launches": K * launches_per_call, "roofline": roofline,
+            "e2e": e2e, "gpu_launches": K * launches_per_call(w.B, greedy), "roofline": roofline,
             "cpu_baseline": cpu, "clocks": clocks.summary(),
             "hbm_gbs": alg / (ms_per_step / 1e3) / 1e9,
             "accept_rate": accept_rate, "mean_accept_len": float(g_len.mean()),
-            "timing": {"region_ms": region_ms, "k1_event_samples": len(k1_ms), "k1_event_every": every,
-                       "k1_ms_median": float(np.median(k1_ms))},
+            "parity": parity,
+            "timing": {"region_ms": region_ms, "k1_event_samples": len(k1_ms),
+                       "k1_pass": "separate pass after the timed region, events around the row-statistics "
+                                  "kernel only"},
+            "per_config": per_config,
         }
         print(json.dumps(line), flush=True)
     if n > 1:
