@@ -59,7 +59,6 @@ METRIC = "verified draft positions/s and achieved HBM GB/s (% of B200 peak), 1 G
 UNIT = "positions/s"
 FALLBACK_HBM_GBS = 6650.0
 MAX_REQUESTS_PER_STATS_LAUNCH = 4096     # mirrors the library's launch split
-MAX_REQUESTS_PER_DRAW_LAUNCH = 65535
 TRAFFIC_FILE = ROOT / "profiles" / "row_stats_traffic.json"
 
 NVML_REASONS = {
@@ -575,7 +574,9 @@ class DeviceWorkload:
         for i in range(samples):
             if self.flush_buf is not None:
                 self.flush_buf.fill_(i)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            # recorded once here so that torch creates the events; the
+            # library records them again around the row-statistics kernel
+            a, b = self.event(), self.event()
             self.step(events=(a, b))
             ev.append((a, b))
         torch.cuda.synchronize()
@@ -638,9 +639,9 @@ def reread_bytes(w, g_len, greedy=False) -> int:
 
 def launches_per_call(B: int, greedy: bool) -> int:
     """Kernels one spec_verify call launches: the row-statistics kernel per
-    block of up to 4096 requests, then the scan-and-draw kernel per block of
-    up to 65535 requests."""
-    return math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + math.ceil(B / MAX_REQUESTS_PER_DRAW_LAUNCH)
+    block of up to 4096 requests, the scan kernel, and (sampling) the draw
+    kernel."""
+    return math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + 1 + (0 if greedy else 1)
 
 
 def config_record(dw, cfg, steps, warmup, k1_samples, peak):

@@ -48,9 +48,11 @@
  * spec_verify_ex and spec_verify_stats is DEVICE memory owned by the caller
  * (spec_verify_host takes host buffers, see there).  The library allocates
  * nothing.  Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL
- * = legacy default stream); results are valid once the stream has reached
- * the call's end.  The workspace needs no initialisation and holds nothing
- * between calls; two calls that run concurrently need separate workspaces.
+ * = legacy default stream) as three kernels -- row statistics, the acceptance
+ * scan and (sampling only) the final draw; results are valid once the stream
+ * has reached the call's end.  The workspace (per-piece row statistics and
+ * the queue of draws) needs no initialisation and holds nothing between
+ * calls; two calls that run concurrently need separate workspaces.
  * The host keeps one small per-device cache of SM count and kernel
  * attributes.
  *
@@ -62,10 +64,11 @@
  * SV_ECUDA.  Values that can only be checked on the device never cause an
  * out-of-bounds access: a request whose draft_lens entry is outside
  * [0, k_max] or whose first L_b drafted ids are outside [0, V) gets
- * out_accept_len = -1 and out_tokens all -1; a request whose statistics were
- * lost to a device-side wait timeout gets out_accept_len = -2 (tests make a
- * wait run out through sv_options.lost_copy_request).  NaN or +inf
- * logits in rows that are read give unspecified (but in-bounds) results.
+ * out_accept_len = -1 and out_tokens all -1; a request whose statistics or
+ * final draw were lost to a device-side wait timeout gets out_accept_len = -2
+ * and out_tokens all -1 (tests make a wait run out through
+ * sv_options.lost_copy_request / lost_draw_request).  NaN or +inf logits in
+ * rows that are read give unspecified (but in-bounds) results.
  */
 #ifndef SPEC_VERIFY_H
 #define SPEC_VERIFY_H
@@ -83,9 +86,9 @@ extern "C" {
 #define SV_API
 #endif
 
-#define SV_ABI_VERSION 1
+#define SV_ABI_VERSION 2
 #define SV_MAX_K 1024      /* largest supported k_max */
-#define SV_MAX_V 393216    /* largest supported vocabulary (8 chunks of 48 Ki) */
+#define SV_MAX_V 393216    /* largest supported vocabulary (96 pieces of 16 KiB in fp32) */
 
 typedef enum { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
 
@@ -114,10 +117,7 @@ typedef enum {
     SV_STATS_AUTO = 0,
     SV_STATS_TMA = 1,    /* cp.async.bulk + mbarrier ring; needs 16-byte aligned rows */
     SV_STATS_VEC16 = 2,  /* 16-byte vector loads; needs 16-byte aligned rows */
-    SV_STATS_SCALAR = 3, /* element loads; any alignment */
-    SV_STATS_FUSED = 4   /* sampling only: the whole step in one persistent launch
-                            (statistics, scan and draw through one bulk-copy ring);
-                            needs 16-byte aligned rows, B <= 4096 */
+    SV_STATS_SCALAR = 3  /* element loads; any alignment */
 } sv_stats_kernel;
 
 typedef struct {
@@ -127,14 +127,22 @@ typedef struct {
     void *event_stats_end;     /* cudaEvent_t recorded just after it, or NULL */
     /* Fault injection for tests of the wait bound; 0 = off.  A value r > 0
      * names request b = r - 1 (0 <= b < B): the bulk-copy statistics kernel
-     * then never issues the copy of the first stage of b's target row 0,
-     * chunk 0.  The wait on that stage runs out after wait_timeout_us, and b
+     * then never issues the copy of the first piece of b's target row 0.
+     * The wait on that stage runs out after wait_timeout_us, and b
      * gets out_accept_len = -2 (so may other requests whose statistics fell
      * to the same CTA after it); the call itself still returns SV_OK and the
      * context stays usable.  Needs the bulk-copy kernel (SV_STATS_TMA, or
      * AUTO on aligned rows): with any other kernel, SV_EUNSUPPORTED. */
     int32_t lost_copy_request;
-    int32_t reserved[7];       /* must be zero */
+    /* Fault injection for tests of the draw kernel's wait bound; 0 = off.  A
+     * value r > 0 names request b = r - 1: if b needs a sampled draw, the
+     * draw kernel never issues the copy of the first piece it stages for b,
+     * so its bounded wait runs out after wait_timeout_us; b (and any later
+     * draw of the same CTA) gets out_accept_len = -2, the call returns SV_OK
+     * and the context stays usable.  No effect on calls without a draw
+     * (greedy, statistics). */
+    int32_t lost_draw_request;
+    int32_t reserved[6];       /* must be zero */
 } sv_options;
 
 /* Bytes of device workspace spec_verify / spec_verify_stats need for this
@@ -258,8 +266,12 @@ SV_API int32_t spec_verify_abi_version(void);
  *   with SV_ESCRATCH before anything is enqueued; use spec_verify then.
  * - The library calls no cudaMalloc / cudaFree or any allocating routine.  The
  *   first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call on a device before capturing a stream.
+ *   (cudaGetSymbolAddress, with that device current) and caches it together
+ *   with the id of the device's current context; make that first call on a
+ *   device before capturing a stream.  If the context is replaced (for
+ *   example cudaDeviceReset, then new work on the device), the next call sees
+ *   a different context id and looks the address up again, so it never uses
+ *   an address of a destroyed context; make that call before any capture too.
  * - All calls share the one array and it keeps the last call's contents (no
  *   part of it needs to start at zero).  Calls whose work overlaps on the GPU
  *   (different streams, or different host threads, without ordering between

@@ -47,7 +47,6 @@ class StatsKernel(enum.IntEnum):
     TMA = 1
     VEC16 = 2
     SCALAR = 3
-    FUSED = 4    # sampling only: statistics, scan and draw in one persistent launch
 
 
 class SpecVerifyError(RuntimeError):
@@ -64,7 +63,8 @@ class _Shape(ctypes.Structure):
 class _Options(ctypes.Structure):
     _fields_ = [("stats_kernel", ctypes.c_int32), ("wait_timeout_us", ctypes.c_int32),
                 ("event_stats_begin", ctypes.c_void_p), ("event_stats_end", ctypes.c_void_p),
-                ("lost_copy_request", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+                ("lost_copy_request", ctypes.c_int32), ("lost_draw_request", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
 
 
 _LIB = None
@@ -191,11 +191,13 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _options(stats_kernel=StatsKernel.AUTO, wait_timeout_us=0, events=None, lost_copy_request=0):
+def _options(stats_kernel=StatsKernel.AUTO, wait_timeout_us=0, events=None, lost_copy_request=0,
+             lost_draw_request=0):
     o = _Options()
     o.stats_kernel = int(stats_kernel)
     o.wait_timeout_us = int(wait_timeout_us)
     o.lost_copy_request = int(lost_copy_request)
+    o.lost_draw_request = int(lost_draw_request)
     if events is not None:
         o.event_stats_begin = events[0].cuda_event
         o.event_stats_end = events[1].cuda_event
@@ -217,13 +219,14 @@ def _logit_shape(target, draft, V):
 
 def spec_verify(target, draft, tokens, lens, uniforms, temperature=1.0, greedy=False, *, V=None,
                 out=None, workspace=None, stream=None, stats_kernel=StatsKernel.AUTO,
-                wait_timeout_us=0, events=None, lost_copy_request=0):
+                wait_timeout_us=0, events=None, lost_copy_request=0, lost_draw_request=0):
     """Verify one batch on the GPU.  Returns ``(accept_len [B] int32,
     tokens [B, k_max+1] int32)`` (device tensors, valid once ``stream`` has
     run).  ``events=(begin, end)`` (torch.cuda.Event, already created)
-    brackets the row-statistics kernel.  ``lost_copy_request`` is the
-    test-only fault injection of ``sv_options`` (1 + the request whose first
-    bulk copy is never issued; 0 = off)."""
+    brackets the row-statistics kernel.  ``lost_copy_request`` and
+    ``lost_draw_request`` are the test-only fault injections of
+    ``sv_options`` (1 + the request whose first bulk copy in the
+    row-statistics / draw kernel is never issued; 0 = off)."""
     torch = _torch()
     B, k_max, V, dt, row_stride = _logit_shape(target, draft, V)
     dev = target.device
@@ -240,7 +243,7 @@ def spec_verify(target, draft, tokens, lens, uniforms, temperature=1.0, greedy=F
     if workspace is None:
         workspace = torch.empty(max(lib.spec_verify_workspace_bytes(ctypes.byref(shape)), 256),
                                 dtype=torch.uint8, device=dev)
-    opts = _options(stats_kernel, wait_timeout_us, events, lost_copy_request)
+    opts = _options(stats_kernel, wait_timeout_us, events, lost_copy_request, lost_draw_request)
     st = lib.spec_verify_ex(
         ctypes.byref(shape), _dev_ptr(target, what="target"), _dev_ptr(draft, what="draft"),
         _dev_ptr(tokens, torch.int32, "draft_tokens"), _dev_ptr(lens, torch.int32, "draft_lens"),

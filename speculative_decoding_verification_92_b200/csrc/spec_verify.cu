@@ -1,6 +1,7 @@
 // spec_verify.cu -- host side of libspecverify.so: argument checks, the
-// chunk plan, launches of K1 (row statistics) and K2 (scan + draw), and the
-// extern "C" entry points declared in include/spec_verify.h.
+// piece plan and workspace layout, launches of K1 (row statistics), K2a
+// (acceptance scan) and K2b (final draw), and the extern "C" entry points
+// declared in include/spec_verify.h.
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -11,8 +12,8 @@
 #include "spec_verify.h"
 #include "sv_common.cuh"
 #include "sv_row_stats.cuh"
+#include "sv_verify_scan.cuh"
 #include "sv_verify_draw.cuh"
-#include "sv_fused.cuh"
 
 namespace sv {
 namespace {
@@ -20,10 +21,6 @@ namespace {
 constexpr int kTmaConsumerWarps = SV_TMA_CONSUMER_WARPS;
 constexpr int kTmaStages = SV_TMA_STAGES;
 constexpr int kLdgThreads = 256;
-// Draw-kernel grid: about SV_DRAW_WAVES waves of kDrawCtasPerSm CTAs per SM.
-#ifndef SV_DRAW_WAVES
-#define SV_DRAW_WAVES 2
-#endif
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 
@@ -37,24 +34,62 @@ DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
 // Fixed scratch of spec_verify_static_scratch (see the header): one array per
-// device, holding the row-statistics partials.  Host code may only use the
-// device address looked up with cudaGetSymbolAddress, cached per device.
+// device, holding the workspace of the same kernels.  Host code may only use
+// the device address looked up with cudaGetSymbolAddress (with the device
+// current), cached per device together with the unique id of the context it
+// was looked up in: when the device's context is replaced (cudaDeviceReset
+// and a new context), the id changes and the address is looked up again.
 static __device__ __align__(256) unsigned char g_static_scratch[SV_STATIC_SCRATCH_BYTES];
-void* g_static_scratch_addr[kMaxDevices];
+
+struct ScratchAddr {
+    void* addr = nullptr;
+    unsigned long long ctx_id = 0;
+};
+ScratchAddr g_static_scratch_addr[kMaxDevices];
+
+// Unique id of the calling thread's current context (driver entry points
+// looked up through the runtime, so the library needs no link to the driver
+// library); 0 when there is none or the driver cannot tell.
+unsigned long long current_context_id() {
+    using GetCurrent = int (*)(void**);
+    using GetId = int (*)(void*, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(f);
+    });
+    if (!get_current || !get_id) return 0;
+    void* ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+    return id;
+}
 
 cudaError_t static_scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const unsigned long long id = current_context_id();
     std::lock_guard<std::mutex> lock(g_dev_mutex);
-    if (!g_static_scratch_addr[dev]) {
+    ScratchAddr& c = g_static_scratch_addr[dev];
+    if (!c.addr || id == 0 || c.ctx_id != id) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_scratch);  // with device `dev` current
         if (e != cudaSuccess) return e;
-        g_static_scratch_addr[dev] = p;
+        c.addr = p;
+        c.ctx_id = current_context_id();                 // the context the lookup made current
     }
-    *out = g_static_scratch_addr[dev];
+    *out = c.addr;
     return cudaSuccess;
 }
 
@@ -83,28 +118,20 @@ cudaError_t allow_smem(Kernel k, size_t bytes) {
 }
 
 struct Plan {
-    int C = 1;       // chunks per row
-    int CE = 8;      // elements per chunk (multiple of 8)
+    int P = 1;       // pieces per row
+    int PE = 4096;   // elements per piece
     int es = 4;      // element size
     int64_t stride = 0;
 };
 
-// Rows are cut into at most kMaxChunks chunks, each a whole number of the
-// row-statistics kernel's bulk-copy stages; a chunk starts on a 16-byte
-// boundary of an aligned row.
+// Rows are cut into pieces of kPieceBytes (the last one ragged); a piece
+// starts on a 16-byte boundary of an aligned row.
 Plan make_plan(const sv_shape& s) {
     Plan p;
     p.es = s.dtype == SV_BF16 ? 2 : 4;
     p.stride = s.row_stride ? s.row_stride : s.V;
-    // A chunk is a whole number of bulk-copy stages, so the row-statistics
-    // ring moves full stages except at the end of each row: the fewest
-    // stages per chunk that keep C <= kMaxChunks.
-    const int64_t row_bytes = int64_t(s.V) * p.es;
-    const int64_t span = int64_t(kMaxChunks) * kStageBytes;
-    int64_t spc = (row_bytes + span - 1) / span;
-    spc = spc < 1 ? 1 : spc;
-    p.CE = static_cast<int>(spc * (kStageBytes / p.es));
-    p.C = static_cast<int>((s.V + p.CE - 1) / p.CE);
+    p.PE = kPieceBytes / p.es;
+    p.P = static_cast<int>((int64_t(s.V) + p.PE - 1) / p.PE);
     return p;
 }
 
@@ -118,21 +145,29 @@ bool shape_ok(const sv_shape* s, sv_status* why) {
     return true;
 }
 
-// Segments of 32 vectors in one chunk (the draw's finest sums).
-int nseg_max_of(const Plan& p) {
-    const int vecs = (p.CE * p.es + 15) / 16;
-    return (vecs + kSegVecs - 1) / kSegVecs;
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Workspace: the row-statistics partials, then the draw queue the scan
+// kernel fills and the draw kernel drains.
+struct WsLayout {
+    size_t partials, ctrl, res_req, one_req, res_cnt, seg, total;
+};
+
+WsLayout ws_layout(const sv_shape& s, const Plan& p) {
+    const size_t B = size_t(s.B);
+    WsLayout l{};
+    size_t off = 0;
+    l.partials = off; off += align256(B * size_t(2 * s.k_max + 1) * size_t(p.P) * sizeof(float2));
+    l.ctrl = off;     off += 256;
+    l.res_req = off;  off += align256(B * sizeof(DrawReq));
+    l.one_req = off;  off += align256(B * sizeof(DrawReq));
+    l.res_cnt = off;  off += align256(B * sizeof(int32_t));
+    l.seg = off;      off += align256(B * size_t(p.P) * kSegsPerPiece * sizeof(float));
+    l.total = off;
+    return l;
 }
 
-// The two-kernel path uses the first part (C partials per row); the fused
-// path lays out W partials per chunk plus its counters, queue and sums.
-size_t workspace_bytes_for(const sv_shape& s, const Plan& p) {
-    const size_t n = size_t(s.B) * size_t(2 * s.k_max + 1) * size_t(p.C) * sizeof(float2);
-    const size_t two_kernel = (n + 255) & ~size_t(255);
-    const size_t fused =
-        fused_layout(s.B, s.k_max, p.C, kTmaConsumerWarps, nseg_max_of(p), p.CE * p.es / kPieceBytes).total;
-    return two_kernel > fused ? two_kernel : fused;
-}
+size_t workspace_bytes_for(const sv_shape& s, const Plan& p) { return ws_layout(s, p).total; }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
@@ -143,7 +178,7 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
         prm.b0 = b0;
         prm.nB = B - b0 < kMaxRequestsPerLaunch ? B - b0 : kMaxRequestsPerLaunch;
         const int rows_max = prm.use_draft ? 2 * prm.k_max + 1 : prm.k_max + 1;
-        const int64_t items_upper = int64_t(prm.nB) * rows_max * prm.C;
+        const int64_t items_upper = int64_t(prm.nB) * rows_max * prm.P;
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         cfg.stream = st;
@@ -188,37 +223,48 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
     return cudaSuccess;
 }
 
+// K2a, one CTA per request, then K2b (sampling), each a programmatic
+// dependent of the kernel before it.
 template <typename T>
-cudaError_t launch_draw(const DrawParams& base, int B, cudaStream_t st) {
-    // A request's cluster has C2 = ceil(C / R) CTAs; R is chosen so that the
-    // whole batch is about SV_DRAW_WAVES waves of CTAs.
-    auto k = verify_draw_kernel<T>;
-    const size_t smem = draw_smem_bytes(base.k_max, base.fast_draw != 0);
-    cudaError_t e = allow_smem(k, smem);
-    if (e != cudaSuccess) return e;
-    for (int b0 = 0; b0 < B; b0 += 65535) {
-        DrawParams prm = base;
-        prm.b0 = b0;
-        const int nB = B - b0 < 65535 ? B - b0 : 65535;
-        const int C2 = (prm.C + prm.R - 1) / prm.R;
+cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, int B, bool draw, const DeviceInfo& dev,
+                             cudaStream_t st) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    {
+        auto k = verify_scan_kernel<T>;
+        const size_t smem = scan_smem_bytes(sp.k_max);
+        cudaError_t e = allow_smem(k, smem);
+        if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[2];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(C2);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        // programmatic dependent of the row-statistics kernel launched just before
-        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[1].val.programmaticStreamSerializationAllowed = 1;
-        cfg.gridDim = dim3(static_cast<unsigned>(C2), static_cast<unsigned>(nB));
-        cfg.blockDim = dim3(kDrawThreads);
+        cfg.gridDim = dim3(static_cast<unsigned>(B));
+        cfg.blockDim = dim3(kScanThreads);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
         cfg.attrs = attr;
-        cfg.numAttrs = 2;
-        if ((e = cudaLaunchKernelEx(&cfg, k, prm)) != cudaSuccess) return e;
+        cfg.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&cfg, k, sp)) != cudaSuccess) return e;
     }
-    return cudaSuccess;
+    if (!draw) return cudaSuccess;
+    auto k = verify_draw_kernel<T>;
+    cudaError_t e = allow_smem(k, kDrawSmemBytes);
+    if (e != cudaSuccess) return e;
+    // persistent: at most one wave of resident CTAs, and no more than the
+    // largest possible number of tasks
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kDrawThreads, kDrawSmemBytes)) != cudaSuccess)
+        return e;
+    per_sm = per_sm < 1 ? 1 : (per_sm > kDrawCtasPerSm ? kDrawCtasPerSm : per_sm);
+    const int64_t cap = int64_t(dev.sm_count) * per_sm;
+    const int64_t max_tasks = int64_t(B) * (dp.P + 1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(max_tasks < cap ? max_tasks : cap));
+    cfg.blockDim = dim3(kDrawThreads);
+    cfg.dynamicSmemBytes = kDrawSmemBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, dp);
 }
 
 struct Call {
@@ -254,22 +300,26 @@ template <typename T>
 sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int variant, bool rows_aligned) {
     const sv_shape& s = *a.shape;
     const bool greedy = a.greedy && !a.stats_only;
+    const WsLayout wl = ws_layout(s, plan);
+    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+    int32_t* ctrl = reinterpret_cast<int32_t*>(ws + wl.ctrl);
     StatsParams sp{};
     sp.target = static_cast<const unsigned char*>(a.target);
     sp.draft = static_cast<const unsigned char*>(a.draft);
     sp.lens = a.lens;
-    sp.partials = static_cast<float2*>(a.workspace);
+    sp.partials = reinterpret_cast<float2*>(ws + wl.partials);
+    sp.ctrl = ctrl;
     sp.k_max = s.k_max;
     sp.V = s.V;
     sp.row_stride = plan.stride;
-    sp.C = plan.C;
-    sp.CE = plan.CE;
+    sp.P = plan.P;
+    sp.PE = plan.PE;
     sp.scale = greedy ? 1.f : static_cast<float>(kLog2e / static_cast<double>(a.temperature));
     sp.use_draft = (a.draft != nullptr && !greedy) ? 1 : 0;
     const int tmo = a.opts ? a.opts->wait_timeout_us : 0;
     sp.timeout_ns = tmo > 0 ? uint64_t(tmo) * 1000ull : kDefaultTimeoutNs;
     const int lost = a.opts ? a.opts->lost_copy_request : 0;
-    sp.lost_copy_partial = lost > 0 ? int64_t(lost - 1) * (2 * s.k_max + 1) * plan.C : -1;
+    sp.lost_copy_partial = lost > 0 ? int64_t(lost - 1) * (2 * s.k_max + 1) * plan.P : -1;
 
     cudaError_t e = cudaSuccess;
     if (a.opts && a.opts->event_stats_begin)
@@ -282,120 +332,60 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
         if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_end), a.stream)) != cudaSuccess)
             return SV_ECUDA;
 
+    ScanParams cp{};
+    cp.target = sp.target;
+    cp.draft = greedy ? nullptr : sp.draft;
+    cp.tokens = a.tokens;
+    cp.lens = a.lens;
+    cp.uniforms = a.uniforms;
+    cp.partials = sp.partials;
+    cp.out_len = a.out_len;
+    cp.out_tokens = a.out_tokens;
+    cp.out_lse_t = a.out_lse_t;
+    cp.out_lse_d = a.out_lse_d;
+    cp.out_p = a.out_p;
+    cp.out_q = a.out_q;
+    cp.out_accept_prob = a.out_accept_prob;
+    cp.out_expected_len = a.out_expected_len;
+    cp.out_first_reject = a.out_first_reject;
+    cp.out_weights = a.out_weights;
+    cp.decay = a.decay;
+    cp.ctrl = ctrl;
+    cp.res_req = reinterpret_cast<DrawReq*>(ws + wl.res_req);
+    cp.one_req = reinterpret_cast<DrawReq*>(ws + wl.one_req);
+    cp.res_cnt = reinterpret_cast<int32_t*>(ws + wl.res_cnt);
+    cp.k_max = s.k_max;
+    cp.V = s.V;
+    cp.row_stride = plan.stride;
+    cp.P = plan.P;
+    cp.PE = plan.PE;
+    cp.scale = sp.scale;
+    cp.greedy = greedy ? 1 : 0;
+    cp.stats_only = a.stats_only ? 1 : 0;
+
     DrawParams dp{};
     dp.target = sp.target;
-    dp.draft = greedy ? nullptr : sp.draft;
-    dp.tokens = a.tokens;
-    dp.lens = a.lens;
-    dp.uniforms = a.uniforms;
+    dp.draft = cp.draft;
     dp.partials = sp.partials;
+    dp.ctrl = ctrl;
+    dp.res_req = cp.res_req;
+    dp.one_req = cp.one_req;
+    dp.res_cnt = cp.res_cnt;
+    dp.seg = reinterpret_cast<float*>(ws + wl.seg);
     dp.out_len = a.out_len;
     dp.out_tokens = a.out_tokens;
-    dp.out_lse_t = a.out_lse_t;
-    dp.out_lse_d = a.out_lse_d;
-    dp.out_p = a.out_p;
-    dp.out_q = a.out_q;
     dp.k_max = s.k_max;
     dp.V = s.V;
     dp.row_stride = plan.stride;
-    dp.C = plan.C;
-    dp.CE = plan.CE;
+    dp.P = plan.P;
+    dp.PE = plan.PE;
     dp.scale = sp.scale;
-    dp.greedy = greedy ? 1 : 0;
-    dp.stats_only = a.stats_only ? 1 : 0;
-    dp.out_accept_prob = a.out_accept_prob;
-    dp.out_expected_len = a.out_expected_len;
-    dp.out_first_reject = a.out_first_reject;
-    dp.out_weights = a.out_weights;
-    dp.decay = a.decay;
     dp.rows_aligned = rows_aligned ? 1 : 0;
-    // the ring pass needs whole pieces per chunk and at most kMaxSegsPerChunk segments
-    const int64_t chunk_bytes = int64_t(plan.CE) * plan.es;
-    dp.fast_draw = (rows_aligned && !greedy && !a.stats_only && chunk_bytes <= kMaxChunkBytesFast &&
-                    chunk_bytes % (int64_t(kPieceVecs) * 16) == 0) ? 1 : 0;
-    {
-        // fewest chunks per CTA that fit the batch in about SV_DRAW_WAVES
-        // waves, then spread evenly: C2 = ceil(C / r) CTAs of ceil(C / C2) chunks
-        const int64_t target_ctas = int64_t(dev.sm_count) * kDrawCtasPerSm * SV_DRAW_WAVES;
-        int64_t r = (int64_t(plan.C) * s.B + target_ctas - 1) / target_ctas;
-        r = r < 1 ? 1 : (r > plan.C ? plan.C : r);
-        const int C2 = static_cast<int>((plan.C + r - 1) / r);
-        dp.R = (plan.C + C2 - 1) / C2;
-    }
-    e = launch_draw<T>(dp, s.B, a.stream);
+    dp.timeout_ns = sp.timeout_ns;
+    const int lost_draw = a.opts ? a.opts->lost_draw_request : 0;
+    dp.lost_draw_b = lost_draw > 0 ? lost_draw - 1 : -1;
+    e = launch_scan_draw<T>(cp, dp, s.B, !greedy && !a.stats_only, dev, a.stream);
     return e == cudaSuccess ? SV_OK : SV_ECUDA;
-}
-
-// Whether the one-launch path can run this call.
-bool fused_ok(const Call& a, const Plan& plan, bool rows_aligned) {
-    const sv_shape& s = *a.shape;
-    const int64_t chunk_bytes = int64_t(plan.CE) * plan.es;
-    return !a.greedy && !a.stats_only && rows_aligned && s.B <= kMaxRequestsPerLaunch && s.k_max >= 0 &&
-           chunk_bytes <= kMaxChunkBytesFast && chunk_bytes % kPieceBytes == 0 && plan.C <= kMaxChunks;
-}
-
-template <typename T>
-sv_status run_fused(const Call& a, const Plan& plan, const DeviceInfo& dev) {
-    const sv_shape& s = *a.shape;
-    const int nseg_max = nseg_max_of(plan);
-    const int P = plan.CE * plan.es / kPieceBytes;   // draw pieces per chunk
-    const FusedLayout l = fused_layout(s.B, s.k_max, plan.C, kTmaConsumerWarps, nseg_max, P);
-    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
-    FusedParams fp{};
-    fp.target = static_cast<const unsigned char*>(a.target);
-    fp.draft = static_cast<const unsigned char*>(a.draft);
-    fp.tokens = a.tokens;
-    fp.lens = a.lens;
-    fp.uniforms = a.uniforms;
-    fp.out_len = a.out_len;
-    fp.out_tokens = a.out_tokens;
-    fp.partials = reinterpret_cast<float2*>(ws + l.partials);
-    fp.state = reinterpret_cast<FusedState*>(ws + l.state);
-    fp.done_items = reinterpret_cast<int32_t*>(ws + l.done_items);
-    fp.draw_done = reinterpret_cast<int32_t*>(ws + l.draw_done);
-    fp.final_flag = reinterpret_cast<int32_t*>(ws + l.final_flag);
-    fp.mbox_ready = reinterpret_cast<int32_t*>(ws + l.mbox_ready);
-    fp.mbox_task = reinterpret_cast<int32_t*>(ws + l.mbox_task);
-    fp.req = reinterpret_cast<FusedReq*>(ws + l.req);
-    fp.segs = reinterpret_cast<float*>(ws + l.segs);
-    fp.piece_tot = reinterpret_cast<float*>(ws + l.piece_tot);
-    fp.P = P;
-    fp.B = s.B;
-    fp.k_max = s.k_max;
-    fp.V = s.V;
-    fp.row_stride = plan.stride;
-    fp.C = plan.C;
-    fp.CE = plan.CE;
-    fp.nseg_max = nseg_max;
-    fp.scale = static_cast<float>(kLog2e / static_cast<double>(a.temperature));
-    const int tmo = a.opts ? a.opts->wait_timeout_us : 0;
-    fp.timeout_ns = tmo > 0 ? uint64_t(tmo) * 1000ull : kDefaultTimeoutNs;
-
-    cudaError_t e = cudaMemsetAsync(ws + l.zero_begin, 0, l.zero_end - l.zero_begin, a.stream);
-    if (e != cudaSuccess) return SV_ECUDA;
-    auto k = verify_fused_kernel<T, kTmaConsumerWarps, kTmaStages>;
-    const size_t smem = FusedSmem<kTmaConsumerWarps, kTmaStages>::bytes(s.B, nseg_max);
-    if ((e = allow_smem(k, smem)) != cudaSuccess) return SV_ECUDA;
-    constexpr int kThreadsF = (kTmaConsumerWarps + 1) * 32;
-    int per_sm = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreadsF, smem)) != cudaSuccess)
-        return SV_ECUDA;
-    per_sm = per_sm < 1 ? 1 : (per_sm > TmaCtasPerSm<T>::value ? TmaCtasPerSm<T>::value : per_sm);
-    const int rows_max = a.draft ? 2 * s.k_max + 1 : s.k_max + 1;
-    const int64_t work = int64_t(s.B) * rows_max * plan.C;
-    int64_t cap = int64_t(dev.sm_count) * per_sm;
-    cap = cap < kMaxFusedGrid ? cap : kMaxFusedGrid;
-    const int64_t grid = work < cap ? (work < 1 ? 1 : work) : cap;
-    fp.mbox_slots = static_cast<int>((int64_t(s.B) * plan.C * P + grid - 1) / grid + 1);
-    if (a.opts && a.opts->event_stats_begin)
-        if (cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_begin), a.stream) != cudaSuccess)
-            return SV_ECUDA;
-    k<<<dim3(static_cast<unsigned>(grid)), dim3(kThreadsF), smem, a.stream>>>(fp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return SV_ECUDA;
-    if (a.opts && a.opts->event_stats_end)
-        if (cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_end), a.stream) != cudaSuccess)
-            return SV_ECUDA;
-    return SV_OK;
 }
 
 sv_status run(const Call& a) {
@@ -403,10 +393,11 @@ sv_status run(const Call& a) {
     if (!shape_ok(a.shape, &why)) return why;
     const sv_shape& s = *a.shape;
     if (a.opts) {
-        for (int i = 0; i < 7; ++i)
+        for (int i = 0; i < 6; ++i)
             if (a.opts->reserved[i] != 0) return SV_EINVAL;
         if (a.opts->lost_copy_request < 0 || a.opts->lost_copy_request > s.B) return SV_EINVAL;
-        if (a.opts->stats_kernel < SV_STATS_AUTO || a.opts->stats_kernel > SV_STATS_FUSED) return SV_EINVAL;
+        if (a.opts->lost_draw_request < 0 || a.opts->lost_draw_request > s.B) return SV_EINVAL;
+        if (a.opts->stats_kernel < SV_STATS_AUTO || a.opts->stats_kernel > SV_STATS_SCALAR) return SV_EINVAL;
         if (a.opts->wait_timeout_us < 0) return SV_EINVAL;
     }
     if (s.B == 0) return SV_OK;
@@ -432,7 +423,6 @@ sv_status run(const Call& a) {
 
     DeviceInfo* dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return SV_ECUDA;
-    if (draw_smem_bytes(s.k_max, true) + 16384 > size_t(dev->max_smem_optin)) return SV_EUNSUPPORTED;
 
     // Kernel choice: the bulk-copy and vector paths need every row start on a
     // 16-byte boundary.
@@ -442,16 +432,10 @@ sv_status run(const Call& a) {
     if (variant == SV_STATS_AUTO) variant = rows_aligned ? SV_STATS_TMA : SV_STATS_SCALAR;
     if ((variant == SV_STATS_TMA || variant == SV_STATS_VEC16) && !rows_aligned) return SV_EINVAL;
     if (a.opts && a.opts->lost_copy_request != 0 && variant != SV_STATS_TMA) return SV_EUNSUPPORTED;
-    if (variant == SV_STATS_FUSED) {
-        if (!fused_ok(a, plan, rows_aligned)) return SV_EINVAL;
-        return s.dtype == SV_BF16 ? run_fused<bf16_bits>(a, plan, *dev) : run_fused<float>(a, plan, *dev);
-    }
 
     return s.dtype == SV_BF16 ? run_typed<bf16_bits>(a, plan, *dev, variant, rows_aligned)
                               : run_typed<float>(a, plan, *dev, variant, rows_aligned);
 }
-
-size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
 struct HostLayout {
     size_t target, draft, tokens, lens, uniforms, out_len, out_tokens, total;

@@ -8,9 +8,15 @@
 
 namespace sv {
 
+// A row is cut into pieces of this many bytes: one bulk-copy stage of the
+// row-statistics kernel, and the unit of work of the draw kernel.
+#ifndef SV_STAGE_BYTES
+#define SV_STAGE_BYTES 16384
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr int kMaxChunks = 8;          // chunks per row == K2 cluster size (portable limit)
+constexpr int kPieceBytes = SV_STAGE_BYTES;
 constexpr int kMaxRequestsPerLaunch = 4096;  // K1 keeps a per-CTA row prefix of this many requests
 
 // ---------------------------------------------------------------------------

@@ -1,33 +1,38 @@
 // sv_row_stats.cuh -- K1, the row-statistics pass.
 //
 // Every row a request uses (target rows 0..L_b, draft rows 0..L_b-1) is cut
-// into C vocabulary chunks of CE elements.  One work item = one (row, chunk);
-// items are dealt round-robin over a persistent grid.  Each item is reduced
-// to one partial:
+// into P pieces of PE elements (16 KiB each, the last one ragged).  The
+// pieces of all used rows, in request order, form one list; CTA x of a grid
+// of G takes the contiguous range [x*N/G, (x+1)*N/G) of the N pieces, so
+// every CTA streams the same number of bytes give or take one piece.  Each
+// piece is reduced to one partial:
 //   sampling: (m, s) with m = max_v t_v, s = sum_v 2^(t_v - m), t_v = z_v * log2(e)/T
 //             (the temperature softmax statistics of step 1 of the rule,
 //             "AI 开始抄自己的作业——而且抄得理直气壮", section "⚡ 投机解码：让草稿先跑，考官殿后")
 //   greedy:   (max z_v, lowest index attaining it)
-// written to partials[(b * (2*k_max+1) + slot) * C + c], slot = i for target
-// row i and k_max+1+i for draft row i.  K2 merges the C partials of a row.
+// written to partials[(b * (2*k_max+1) + slot) * P + piece], slot = i for
+// target row i and k_max+1+i for draft row i.  The scan kernel merges the P
+// partials of a row; the draw kernel uses the pieces as its units of work.
 //
 // Variants:
-//   row_stats_tma_kernel  one producer warp streams each item through a ring
-//                         of shared-memory stages with 1-D cp.async.bulk
-//                         copies completing on mbarriers; consumer warps
-//                         reduce from shared memory.  Needs 16-byte aligned
-//                         rows.  Waits are bounded; a timed-out CTA marks its
-//                         remaining items with NaN partials.
-//   row_stats_ldg_kernel  the same item schedule with 16-byte vector loads
-//                         (aligned rows) or element loads (any alignment).
+//   row_stats_tma_kernel  one producer warp streams the pieces through a ring
+//                         of shared-memory stages (one piece per stage) with
+//                         1-D cp.async.bulk copies completing on mbarriers;
+//                         consumer warps fold the stage and leave one
+//                         (m, s) per thread in shared memory, which the
+//                         producer warp merges into the piece's partial before
+//                         it refills the stage.  Needs 16-byte aligned rows.
+//                         Waits are bounded; after a timeout the CTA writes
+//                         NaN partials for the rest of its range.
+//   row_stats_ldg_kernel  the same piece ranges with 16-byte vector loads
+//                         (aligned rows) or element loads (any alignment) and
+//                         a block reduction per piece.
 #pragma once
 
 #include "sv_common.cuh"
 
-// Ring geometry of the bulk-copy variant (compile-time; defaults tuned on B200).
-#ifndef SV_STAGE_BYTES
-#define SV_STAGE_BYTES 16384
-#endif
+// Ring geometry of the bulk-copy variant (compile-time; defaults tuned on B200;
+// the stage size is SV_STAGE_BYTES of sv_common.cuh).
 #ifndef SV_TMA_CONSUMER_WARPS
 #define SV_TMA_CONSUMER_WARPS 4
 #endif
@@ -50,28 +55,33 @@
 
 namespace sv {
 
+// One piece = one ring stage of the bulk-copy variant.
+constexpr int kStageBytes = kPieceBytes;
+
 struct StatsParams {
     const unsigned char* target;  // [B][k_max+1][row_stride]
     const unsigned char* draft;   // [B][k_max][row_stride] or null
     const int32_t* lens;          // [B] or null (all k_max)
-    float2* partials;             // [B][2*k_max+1][C]
+    float2* partials;             // [B][2*k_max+1][P]
+    int32_t* ctrl;                // the draw kernels' list counters: zeroed by block 0 of the
+                                  // launch with b0 == 0 (null: nothing to zero)
     int32_t b0;                   // first request handled by this launch
     int32_t nB;                   // requests handled by this launch (<= kMaxRequestsPerLaunch)
     int32_t k_max;
     int32_t V;
     int64_t row_stride;           // elements
-    int32_t C;                    // chunks per row
-    int32_t CE;                   // elements per chunk, multiple of 8
+    int32_t P;                    // pieces per row
+    int32_t PE;                   // elements per piece (kPieceBytes / element size)
     float scale;                  // log2(e) / T
     int32_t use_draft;            // draft rows are part of the work
     uint64_t timeout_ns;          // bound on each barrier wait (TMA variant)
-    int64_t lost_copy_partial;    // test fault injection: this item's first stage is never copied; -1 = off
+    int64_t lost_copy_partial;    // test fault injection: this piece is never copied; -1 = off
 };
 
 struct ItemDesc {
     const unsigned char* row;     // first byte of the row
     int64_t partial_idx;
-    int32_t e0, e1;               // element range of the chunk
+    int32_t e0, e1;               // element range of the piece
 };
 
 __device__ __forceinline__ int clamp_len(const StatsParams& p, int b) {
@@ -131,10 +141,11 @@ __device__ void build_row_prefix(const StatsParams& p, int* row_start, int* scra
     __syncthreads();
 }
 
+// Piece `item` of the list: row g = item / P of the used rows, piece item % P.
 template <typename T>
 __device__ __forceinline__ ItemDesc decode_item(const StatsParams& p, const int* row_start, int64_t item) {
-    const int64_t g = item / p.C;
-    const int c = static_cast<int>(item - g * p.C);
+    const int64_t g = item / p.P;
+    const int c = static_cast<int>(item - g * p.P);
     int lo = 0, hi = p.nB;  // row_start[lo] <= g < row_start[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -155,10 +166,16 @@ __device__ __forceinline__ ItemDesc decode_item(const StatsParams& p, const int*
         slot = p.k_max + 1 + i;
         d.row = p.draft + ((int64_t)b * p.k_max + i) * p.row_stride * Logit<T>::kSize;
     }
-    d.partial_idx = ((int64_t)b * (2 * p.k_max + 1) + slot) * p.C + c;
-    d.e0 = c * p.CE;
-    d.e1 = min(p.V, d.e0 + p.CE);
+    d.partial_idx = ((int64_t)b * (2 * p.k_max + 1) + slot) * p.P + c;
+    d.e0 = c * p.PE;
+    d.e1 = min(p.V, d.e0 + p.PE);
     return d;
+}
+
+// This CTA's contiguous range [*lo, *hi) of the piece list.
+__device__ __forceinline__ void piece_range(int64_t total, int64_t* lo, int64_t* hi) {
+    *lo = total * blockIdx.x / gridDim.x;
+    *hi = total * (blockIdx.x + 1) / gridDim.x;
 }
 
 // Per-thread accumulators -----------------------------------------------------
@@ -196,6 +213,7 @@ template <> struct Acc<false> {
         if (m == -INFINITY) return;
         ms = MS{m, ms.s * ex2_approx(ms.m - m) + ex2_approx(t - m)};
     }
+    __device__ __forceinline__ float2 as_float2() const { return make_float2(ms.m, ms.s); }
 };
 
 template <> struct Acc<true> {
@@ -204,6 +222,7 @@ template <> struct Acc<true> {
     __device__ __forceinline__ void take(float z, int idx) {
         if (z > vi.v || (z == vi.v && idx < vi.i)) vi = VI{z, idx};
     }
+    __device__ __forceinline__ float2 as_float2() const { return make_float2(vi.v, __int_as_float(vi.i)); }
 };
 
 // Fold K 16-byte vectors of raw logits into a sampling accumulator.  The
@@ -261,7 +280,7 @@ __device__ __forceinline__ void fold_vectors(Acc<false>& acc, const uint4 (&v)[K
 
 // Fold only the first `nv` (0 <= nv <= K) of K vectors: one fold with a
 // compile-time count per possible nv, so no ex2 is spent on absent elements
-// (the partial stage or batch at the end of each item).
+// (the partial stage at the end of each row).
 template <typename T, int K, int N>
 __device__ __forceinline__ void fold_prefix(Acc<false>& acc, const uint4 (&v)[K], float scale) {
     uint4 part[N];
@@ -293,15 +312,43 @@ __device__ __forceinline__ uint4 neg_inf_vector() {
     return make_uint4(x, x, x, x);
 }
 
-// Reduce the reducing threads' accumulators and let thread 0 write the
-// partial (a NaN pair when any thread lost its data to a wait timeout).
-// `red` holds 3 * kWarps floats for this item (double-buffered by the
-// caller); `bar_id`/`nthreads` name the barrier of the reducing threads.
+// Merge 32 x kPer per-thread partials (one warp, lane l holding parts[l + 32 k])
+// into one; lane 0 gets the result.  Sampling: max first, then every sum
+// rescaled once; greedy: larger value, then lower index.
+template <bool kGreedy, int kPer>
+__device__ __forceinline__ float2 warp_merge_parts(const float2 (&v)[kPer]) {
+    if constexpr (kGreedy) {
+        VI best{v[0].x, __float_as_int(v[0].y)};
+#pragma unroll
+        for (int k = 1; k < kPer; ++k) best = vi_better(best, VI{v[k].x, __float_as_int(v[k].y)});
+        best = warp_merge_vi(best);
+        return make_float2(best.v, __int_as_float(best.i));
+    } else {
+        float m = v[0].x;
+#pragma unroll
+        for (int k = 1; k < kPer; ++k) m = fmaxf(m, v[k].x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float s = 0.f;
+        if (m != -INFINITY) {
+#pragma unroll
+            for (int k = 0; k < kPer; ++k)
+                if (v[k].x != -INFINITY) s = fmaf(v[k].y, ex2_approx(v[k].x - m), s);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        return m == -INFINITY ? make_float2(-INFINITY, 0.f) : make_float2(m, s);
+    }
+}
+
+// Block reduction of the reducing threads' accumulators for the element-load
+// variant; thread 0 writes the partial.  `red` holds 2 * kWarps floats for
+// this item (double-buffered by the caller); `bar_id`/`nthreads` name the
+// barrier of the reducing threads.
 template <bool kGreedy, int kWarps>
 __device__ __forceinline__ void reduce_and_store(Acc<kGreedy>& acc, float* red, int bar_id, int nthreads,
-                                                 float2* out, bool failed) {
+                                                 float2* out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const bool warp_failed = __any_sync(0xffffffffu, failed);
     float a, b;
     if constexpr (kGreedy) {
         VI v = warp_merge_vi(acc.vi);
@@ -313,25 +360,21 @@ __device__ __forceinline__ void reduce_and_store(Acc<kGreedy>& acc, float* red, 
         b = v.s;
     }
     if (lane == 0) {
-        red[3 * warp] = a;
-        red[3 * warp + 1] = b;
-        red[3 * warp + 2] = warp_failed ? 1.f : 0.f;
+        red[2 * warp] = a;
+        red[2 * warp + 1] = b;
     }
     named_barrier_sync(bar_id, nthreads);
     if (threadIdx.x == 0) {
-        bool any_failed = false;
-        for (int w = 0; w < kWarps; ++w) any_failed |= red[3 * w + 2] != 0.f;
         float2 r;
         if constexpr (kGreedy) {
             VI t{red[0], __float_as_int(red[1])};
-            for (int w = 1; w < kWarps; ++w) t = vi_better(t, VI{red[3 * w], __float_as_int(red[3 * w + 1])});
+            for (int w = 1; w < kWarps; ++w) t = vi_better(t, VI{red[2 * w], __float_as_int(red[2 * w + 1])});
             r = make_float2(t.v, __int_as_float(t.i));
         } else {
             MS t{red[0], red[1]};
-            for (int w = 1; w < kWarps; ++w) t = ms_merge(t, MS{red[3 * w], red[3 * w + 1]});
+            for (int w = 1; w < kWarps; ++w) t = ms_merge(t, MS{red[2 * w], red[2 * w + 1]});
             r = make_float2(t.m, t.s);
         }
-        if (any_failed) r = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
         *out = r;
     }
 }
@@ -350,10 +393,15 @@ __device__ __forceinline__ void fold_vector(Acc<kGreedy>& acc, const uint4& w, i
     }
 }
 
+__device__ __forceinline__ void zero_ctrl(const StatsParams& p) {
+    if (p.ctrl && p.b0 == 0 && blockIdx.x == 0 && threadIdx.x == 0) {
+        p.ctrl[0] = 0;
+        p.ctrl[1] = 0;
+    }
+}
+
 // ============================================================================
 // TMA bulk-copy variant.
-
-constexpr int kStageBytes = SV_STAGE_BYTES;
 
 template <typename T>
 struct TmaCtasPerSm {
@@ -361,30 +409,44 @@ struct TmaCtasPerSm {
 };
 
 struct StageMeta {
-    const unsigned char* tail;  // first ragged-tail element (row's last chunk), or null
+    const unsigned char* tail;  // first ragged-tail element (row's last piece), or null
     int64_t partial_idx;
     int32_t elem0;              // row index of the stage's first element
     int32_t n_bytes;            // bytes delivered by the bulk copy (multiple of 16)
     int32_t tail_n;             // ragged-tail elements (< 16 / sizeof element)
-    int32_t flags;              // 1: first stage of the item, 2: last stage of the item
+    int32_t pad;
 };
 
 template <int kConsumerWarps, int kStages>
 struct TmaSmem {
     static constexpr size_t kMetaOff = size_t(kStages) * kStageBytes;
     static constexpr size_t kBarOff = kMetaOff + sizeof(StageMeta) * kStages;
-    static constexpr size_t kMiscOff = kBarOff + 16 * kStages;          // full[], empty[]
-    static constexpr size_t kRedOff = kMiscOff + 4 * 64;                // misc ints
-    static constexpr size_t kRowOff = kRedOff + 4 * 6 * kConsumerWarps;  // red[2][3*warps]
+    static constexpr size_t kMiscOff = kBarOff + 16 * kStages;                         // full[], empty[]
+    static constexpr size_t kPartOff = kMiscOff + 4 * 64;                              // misc ints
+    static constexpr size_t kRowOff = kPartOff + 8 * size_t(kStages) * kConsumerWarps * 32;  // part[stage][thread]
     static size_t bytes(int nB) { return kRowOff + 4 * size_t(nB + 1); }
 };
+
+// Bounded wait that also gives up as soon as *abort_flag is set.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                                   const volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > timeout_ns) return false;
+    }
+}
 
 template <typename T, bool kGreedy, int kConsumerWarps, int kStages>
 __global__ void __launch_bounds__((kConsumerWarps + 1) * 32, TmaCtasPerSm<T>::value)
 row_stats_tma_kernel(const StatsParams p) {
     constexpr int kConsumers = kConsumerWarps * 32;
     constexpr int kThreads = kConsumers + 32;
-    constexpr int kVecPerThread = (kStageBytes / 16 + kConsumers - 1) / kConsumers;
+    constexpr int kVecPerThread = kStageBytes / 16 / kConsumers;
+    static_assert(kStageBytes % (16 * kConsumers) == 0, "a stage must split evenly over the consumers");
+    constexpr int kPartsPerLane = kConsumers / 32;
     using L = TmaSmem<kConsumerWarps, kStages>;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char* stage_buf = smem;
@@ -393,10 +455,11 @@ row_stats_tma_kernel(const StatsParams p) {
     uint64_t* empty = full + kStages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff);
     int* scan_scratch = reinterpret_cast<int*>(smem + L::kMiscOff) + 8;
-    float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+    float2* part = reinterpret_cast<float2*>(smem + L::kPartOff);   // [kStages][kConsumers]
     int* row_start = reinterpret_cast<int*>(smem + L::kRowOff);
 
     const int tid = threadIdx.x;
+    zero_ctrl(p);
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full + s, 1);
@@ -406,145 +469,156 @@ row_stats_tma_kernel(const StatsParams p) {
         fence_mbar_init();
     }
     build_row_prefix<kThreads>(p, row_start, scan_scratch);  // ends with __syncthreads
-    const int64_t total_items = (int64_t)row_start[p.nB] * p.C;
+    int64_t lo, hi;
+    piece_range((int64_t)row_start[p.nB] * p.P, &lo, &hi);
 
     if (tid >= kConsumers) {
         // ----------------------------- producer warp -----------------------------
+        // Issues piece `next` into stage (next - lo) % kStages while the ring
+        // has room; otherwise waits until the consumers have released the
+        // oldest piece in flight, merges their per-thread partials of it and
+        // stores the piece's partial.  Stage s receives its r-th piece in
+        // round r; the consumers' release of it is the r-th completion of
+        // empty[s] (parity r & 1), the copy's arrival the r-th of full[s].
         const int lane = tid - kConsumers;
-        int slot = 0;               // ring position of the next stage
-        uint32_t phase = 0;         // parity of the ring round in progress
-        bool wrapped = false;       // the ring has been filled once
-        uint32_t last_phase[kStages];
+        int64_t next = lo, merged = lo;
+        int last_round[kStages];    // round of the last copy issued into each stage, -1 = none
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) last_phase[s] = 0xffffffffu;
+        for (int s = 0; s < kStages; ++s) last_round[s] = -1;
         bool stop = false;
-        for (int64_t item = blockIdx.x; item < total_items && !stop; item += gridDim.x) {
-            const ItemDesc d = decode_item<T>(p, row_start, item);
-            const int64_t bytes_all = int64_t(d.e1 - d.e0) * Logit<T>::kSize;
-            const int64_t tma_bytes = bytes_all & ~int64_t(15);
-            const int tail_n = static_cast<int>((bytes_all - tma_bytes) / Logit<T>::kSize);
-            const int nsub = tma_bytes == 0 ? 1 : static_cast<int>((tma_bytes + kStageBytes - 1) / kStageBytes);
-            const unsigned char* src0 = d.row + int64_t(d.e0) * Logit<T>::kSize;
-            for (int sub = 0; sub < nsub; ++sub) {
+        while (merged < hi) {
+            if (next < hi && next - merged < kStages) {
+                const int64_t k = next - lo;
+                const int slot = static_cast<int>(k % kStages);
+                const int round = static_cast<int>(k / kStages);
                 if (lane == 0) {
-                    bool ok = true;
-                    if (wrapped) ok = mbar_wait_bounded(empty + slot, phase ^ 1u, p.timeout_ns);
-                    if (!ok) *abort_flag = 1;
-                    if (*abort_flag) {
-                        stop = true;
-                    } else if (sub == 0 && d.partial_idx == p.lost_copy_partial) {
+                    const ItemDesc d = decode_item<T>(p, row_start, next);
+                    const int64_t bytes_all = int64_t(d.e1 - d.e0) * Logit<T>::kSize;
+                    const int n = static_cast<int>(bytes_all & ~int64_t(15));
+                    const int tail_n = static_cast<int>((bytes_all - n) / Logit<T>::kSize);
+                    const unsigned char* src = d.row + int64_t(d.e0) * Logit<T>::kSize;
+                    if (d.partial_idx == p.lost_copy_partial) {
                         // injected fault: the stage is neither armed nor copied, so
-                        // the consumers' bounded wait on it runs out; last_phase[slot]
-                        // keeps the previous (completed) phase for the drain below
+                        // the consumers' bounded wait on it runs out
                     } else {
-                        const int64_t off = int64_t(sub) * kStageBytes;
-                        const int64_t left = tma_bytes - off;
-                        const int n = static_cast<int>(left < kStageBytes ? left : int64_t(kStageBytes));
                         StageMeta m;
-                        m.tail = tail_n ? src0 + tma_bytes : nullptr;
+                        m.tail = tail_n ? src + n : nullptr;
                         m.partial_idx = d.partial_idx;
-                        m.elem0 = d.e0 + static_cast<int>(off / Logit<T>::kSize);
-                        m.n_bytes = n > 0 ? n : 0;
+                        m.elem0 = d.e0;
+                        m.n_bytes = n;
                         m.tail_n = tail_n;
-                        m.flags = (sub == 0 ? 1 : 0) | (sub == nsub - 1 ? 2 : 0);
+                        m.pad = 0;
                         meta[slot] = m;
-                        last_phase[slot] = phase;
+#pragma unroll
+                        for (int s = 0; s < kStages; ++s)
+                            if (s == slot) last_round[s] = round;
                         if (n > 0) {
                             mbar_arrive_expect_tx(full + slot, static_cast<uint32_t>(n));
-                            bulk_copy_g2s(stage_buf + size_t(slot) * kStageBytes, src0 + off,
-                                          static_cast<uint32_t>(n), full + slot);
+                            bulk_copy_g2s(stage_buf + size_t(slot) * kStageBytes, src, static_cast<uint32_t>(n),
+                                          full + slot);
                         } else {
                             mbar_arrive(full + slot);
                         }
                     }
                 }
-                stop = __shfl_sync(0xffffffffu, stop, 0);
-                if (stop) break;
-                if (++slot == kStages) {
-                    slot = 0;
-                    phase ^= 1u;
-                    wrapped = true;
-                }
+                ++next;
+                continue;
             }
+            const int64_t k = merged - lo;
+            const int slot = static_cast<int>(k % kStages);
+            const int round = static_cast<int>(k / kStages);
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait_or_abort(empty + slot, static_cast<uint32_t>(round & 1), p.timeout_ns,
+                                                   abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                if (lane == 0) *abort_flag = 1;
+                stop = true;
+                break;
+            }
+            float2 v[kPartsPerLane];
+            const float2* ps = part + slot * kConsumers;
+#pragma unroll
+            for (int i = 0; i < kPartsPerLane; ++i) v[i] = ps[lane + 32 * i];
+            const float2 r = warp_merge_parts<kGreedy, kPartsPerLane>(v);
+            if (lane == 0) p.partials[meta[slot].partial_idx] = r;
+            ++merged;
         }
-        // Wait until the consumers are done, then (only after a timeout) make
-        // sure no copy issued by this CTA is still in flight before exiting.
+        if (stop) {
+            // the pieces left unmerged get NaN partials: the scan kernel reports
+            // their requests with out_accept_len = -2
+            const float nan = __int_as_float(0x7fc00000);
+            for (int64_t it = merged + lane; it < hi; it += 32)
+                p.partials[decode_item<T>(p, row_start, it).partial_idx] = make_float2(nan, nan);
+        }
+        // Wait until the consumers are done, then make sure no copy issued by
+        // this CTA is still in flight before exiting (after a timeout).
         named_barrier_sync(2, kThreads);
-        if (lane == 0 && *abort_flag) {
+        if (lane == 0 && stop) {
+#pragma unroll
             for (int s = 0; s < kStages; ++s)
-                if (last_phase[s] != 0xffffffffu) (void)mbar_wait_bounded(full + s, last_phase[s], p.timeout_ns);
+                if (last_round[s] >= 0)
+                    (void)mbar_wait_bounded(full + s, static_cast<uint32_t>(last_round[s] & 1), p.timeout_ns);
         }
         return;
     }
 
     // ------------------------------- consumer warps -------------------------------
-    // Every consumer thread runs the reduction of every item exactly once, so
-    // the named barrier 1 stays in step even after a timeout; wait outcomes are
-    // made warp-uniform with __all_sync before anyone acts on them.
-    Acc<kGreedy> acc;
-    int slot = 0;          // ring position of the next stage
-    uint32_t phase = 0;    // parity of the ring round in progress
-    int parity_item = 0;
-    for (int64_t item = blockIdx.x; item < total_items; item += gridDim.x, parity_item ^= 1) {
+    // Each piece: wait for its stage, fold it (plus the row's ragged tail on
+    // the row's last piece), leave this thread's partial in part[stage][tid]
+    // and release the stage.  A failed wait is made warp-uniform; the warp
+    // then leaves the loop (the producer writes the NaN partials).
+    const int lane = tid & 31;
+    for (int64_t piece = lo; piece < hi; ++piece) {
+        const int64_t k = piece - lo;
+        const int slot = static_cast<int>(k % kStages);
+        const uint32_t parity = static_cast<uint32_t>((k / kStages) & 1);
+        bool ok = !*abort_flag && mbar_wait_or_abort(full + slot, parity, p.timeout_ns, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+            if (lane == 0) *abort_flag = 1;
+            break;
+        }
+        const StageMeta m = meta[slot];
+        const unsigned char* buf = stage_buf + size_t(slot) * kStageBytes;
+        const int nvec = m.n_bytes >> 4;
+        Acc<kGreedy> acc;
         acc.reset();
-        bool failed = __any_sync(0xffffffffu, *abort_flag != 0);  // warp-uniform
-        int64_t partial_idx = -1;
-        while (!failed) {
-            bool ok = !*abort_flag && mbar_wait_bounded(full + slot, phase, p.timeout_ns);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) {
-                *abort_flag = 1;
-                failed = true;
-                break;
-            }
-            const StageMeta m = meta[slot];
-            partial_idx = m.partial_idx;
-            const unsigned char* buf = stage_buf + size_t(slot) * kStageBytes;
-            const int nvec = m.n_bytes >> 4;
-            if constexpr (kGreedy) {
+        if constexpr (kGreedy) {
 #pragma unroll
-                for (int k = 0; k < kVecPerThread; ++k) {
-                    const int v = tid + k * kConsumers;
-                    if (v < nvec) fold_vector<T, true>(acc, ld_shared_v4(buf + 16 * v), m.elem0 + v * Logit<T>::kPerVec, 0.f);
-                }
+            for (int kk = 0; kk < kVecPerThread; ++kk) {
+                const int v = tid + kk * kConsumers;
+                if (v < nvec)
+                    fold_vector<T, true>(acc, ld_shared_v4(buf + 16 * v), m.elem0 + v * Logit<T>::kPerVec, 0.f);
+            }
+        } else {
+            uint4 vv[kVecPerThread];
+            if (nvec == kVecPerThread * kConsumers) {  // full stage: no guards
+#pragma unroll
+                for (int kk = 0; kk < kVecPerThread; ++kk) vv[kk] = ld_shared_v4(buf + 16 * (tid + kk * kConsumers));
+                fold_vectors<T, kVecPerThread>(acc, vv, p.scale);
             } else {
-                uint4 vv[kVecPerThread];
-                if (nvec == kVecPerThread * kConsumers) {  // full stage: no guards
 #pragma unroll
-                    for (int k = 0; k < kVecPerThread; ++k) vv[k] = ld_shared_v4(buf + 16 * (tid + k * kConsumers));
-                    fold_vectors<T, kVecPerThread>(acc, vv, p.scale);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < kVecPerThread; ++k) {
-                        const int v = tid + k * kConsumers;
-                        vv[k] = v < nvec ? ld_shared_v4(buf + 16 * v) : make_uint4(0, 0, 0, 0);
-                    }
-                    const int nv = nvec > tid ? (nvec - tid + kConsumers - 1) / kConsumers : 0;
-                    fold_vectors_count<T, kVecPerThread>(acc, vv, nv, p.scale);
+                for (int kk = 0; kk < kVecPerThread; ++kk) {
+                    const int v = tid + kk * kConsumers;
+                    vv[kk] = v < nvec ? ld_shared_v4(buf + 16 * v) : make_uint4(0, 0, 0, 0);
                 }
-            }
-            __syncwarp();
-            if ((tid & 31) == 0) mbar_arrive(empty + slot);
-            if (++slot == kStages) {
-                slot = 0;
-                phase ^= 1u;
-            }
-            if (m.flags & 2) {
-                if (m.tail && tid < m.tail_n) {
-                    const float z = Logit<T>::load(m.tail, tid);
-                    const int idx = m.elem0 + (m.n_bytes / Logit<T>::kSize) + tid;
-                    if constexpr (kGreedy) acc.take(z, idx);
-                    else acc.fold1(z * p.scale);
-                }
-                break;
+                const int nv = nvec > tid ? (nvec - tid + kConsumers - 1) / kConsumers : 0;
+                fold_vectors_count<T, kVecPerThread>(acc, vv, nv, p.scale);
             }
         }
-        if (failed) partial_idx = decode_item<T>(p, row_start, item).partial_idx;
-        reduce_and_store<kGreedy, kConsumerWarps>(acc, red + parity_item * 3 * kConsumerWarps, 1, kConsumers,
-                                                 p.partials + partial_idx, failed);
+        if (m.tail && tid < m.tail_n) {
+            const float z = Logit<T>::load(m.tail, tid);
+            const int idx = m.elem0 + (m.n_bytes / Logit<T>::kSize) + tid;
+            if constexpr (kGreedy) acc.take(z, idx);
+            else acc.fold1(z * p.scale);
+        }
+        part[slot * kConsumers + tid] = acc.as_float2();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + slot);  // release: the partials above are visible to the producer
     }
     named_barrier_sync(2, kThreads);
-    // this CTA is done: the dependent draw kernel may start its prologue here
+    // this CTA is done: the dependent scan kernel may start its prologue here
     if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
 }
 
@@ -558,12 +632,14 @@ row_stats_ldg_kernel(const StatsParams p) {
     constexpr int kUnroll = SV_LDG_UNROLL;
     extern __shared__ __align__(16) int ldg_row_start[];
     __shared__ int scan_scratch[32];
-    __shared__ float red[2][3 * kWarps];
+    __shared__ float red[2][2 * kWarps];
+    zero_ctrl(p);
     build_row_prefix<kThreads>(p, ldg_row_start, scan_scratch);
-    const int64_t total_items = (int64_t)ldg_row_start[p.nB] * p.C;
+    int64_t lo, hi;
+    piece_range((int64_t)ldg_row_start[p.nB] * p.P, &lo, &hi);
     const int tid = threadIdx.x;
     int parity_item = 0;
-    for (int64_t item = blockIdx.x; item < total_items; item += gridDim.x, parity_item ^= 1) {
+    for (int64_t item = lo; item < hi; ++item, parity_item ^= 1) {
         const ItemDesc d = decode_item<T>(p, ldg_row_start, item);
         Acc<kGreedy> acc;
         acc.reset();
@@ -613,7 +689,7 @@ row_stats_ldg_kernel(const StatsParams p) {
                 else acc.fold1(z * p.scale);
             }
         }
-        reduce_and_store<kGreedy, kWarps>(acc, red[parity_item], 1, kThreads, p.partials + d.partial_idx, false);
+        reduce_and_store<kGreedy, kWarps>(acc, red[parity_item], 1, kThreads, p.partials + d.partial_idx);
     }
     __syncthreads();
     if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");

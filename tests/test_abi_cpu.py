@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 8, names
     for name in names:
         assert hasattr(lib, name), f"{name} is declared in include/ but not exported"
-    assert sv.abi_version() == 1
+    assert sv.abi_version() == 2
 
 
 def test_status_strings():
@@ -39,36 +39,23 @@ def test_status_strings():
     assert lib.spec_verify_status_string(99) == b"unknown status"
 
 
-STAGE_BYTES, MAX_CHUNKS = 16384, 8
-
-
-def plan_chunks(V, es):
-    """Chunks are whole 16 KiB stages, as few per chunk as keep C <= 8."""
-    spc = max(1, -(-V * es // (MAX_CHUNKS * STAGE_BYTES)))
-    ce = spc * STAGE_BYTES // es
-    return -(-V // ce), ce
+PIECE_BYTES = 16384
 
 
 def a256(n):
     return (n + 255) // 256 * 256
 
 
-def fused_bytes(B, k, C, CE, es, W=4):
-    """The one-launch layout: W partials per chunk, counters, task queue,
-    per-request records (48 B) and one sum per 32-vector segment."""
-    nseg = -(-(CE * es // 16) // 32)
-    P = CE * es // 8192               # draw pieces (one 8 KiB ring stage per row) per chunk
-    mbox = B * C * P + 2 * 1024       # per-CTA task mailboxes
-    return (a256(8 * B * (2 * k + 1) * C * W) + a256(32) + 3 * a256(4 * B) + a256(4 * mbox)
-            + a256(4 * mbox) + a256(48 * B) + a256(4 * B * C * nseg) + a256(4 * B * C * P * W))
-
-
 @pytest.mark.parametrize("B,k,V,dt", [(64, 8, 151936, sv.BF16), (256, 12, 128256, sv.F32),
                                       (4, 4, 1000, sv.F32), (3, 0, 5, sv.BF16), (0, 3, 100, sv.F32)])
 def test_workspace_bytes(B, k, V, dt):
+    """Rows are cut into 16 KiB pieces (P per row); the workspace holds one
+    8-byte partial per (request, row slot, piece), a 256-byte control block,
+    two queues of 48-byte draw records, one counter per request and 32
+    segment sums per (request, piece)."""
     es = 2 if dt == sv.BF16 else 4
-    C, CE = plan_chunks(V, es)
-    want = max(a256(B * (2 * k + 1) * C * 8), fused_bytes(B, k, C, CE, es))
+    P = -(-V * es // PIECE_BYTES)
+    want = (a256(8 * B * (2 * k + 1) * P) + 256 + 2 * a256(48 * B) + a256(4 * B) + a256(4 * 32 * B * P))
     assert sv.workspace_bytes(B, k, V, dt) == want
 
 
@@ -121,15 +108,19 @@ def test_bad_options():
     o = _Options()
     o.reserved[3] = 1
     assert call(opts=o) == Status.EINVAL
-    o = _Options()
-    o.stats_kernel = 7
-    assert call(opts=o) == Status.EINVAL
+    for kernel in (4, 7, -1):               # only AUTO, TMA, VEC16 and SCALAR exist
+        o = _Options()
+        o.stats_kernel = kernel
+        assert call(opts=o) == Status.EINVAL
     o = _Options()
     o.wait_timeout_us = -5
     assert call(opts=o) == Status.EINVAL
     for r in (-1, 5):                      # names no request of the B = 4 batch
         o = _Options()
         o.lost_copy_request = r
+        assert call(opts=o) == Status.EINVAL
+        o = _Options()
+        o.lost_draw_request = r
         assert call(opts=o) == Status.EINVAL
 
 

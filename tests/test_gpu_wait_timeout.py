@@ -53,3 +53,44 @@ def test_lost_copy_needs_the_bulk_copy_kernel():
         with pytest.raises(sv.SpecVerifyError):
             sv.spec_verify(d["target"], d["draft"], d["tokens"], d["lens"], d["uniforms"], V=w.V,
                            stats_kernel=kernel, lost_copy_request=1)
+
+
+def draw_victims(clean_len, w):
+    """One request whose draw is a redraw after a rejection (j < L) and one
+    whose draw is the bonus token (j == L)."""
+    L = w.draft_lens
+    resid = [b for b in range(w.B) if 0 <= clean_len[b] < L[b]]
+    bonus = [b for b in range(w.B) if clean_len[b] == L[b]]
+    return resid[:1] + bonus[:1]
+
+
+@pytest.mark.parametrize("V,dtype,mode,misalign", [(1000, F32, "logits", False), (151936, BF16, "logits", False),
+                                                   (151936, BF16, "ids", False), (4099, F32, "logits", True)])
+def test_lost_draw_copy_times_out_and_the_context_stays_usable(V, dtype, mode, misalign):
+    """The draw kernel's waits on its own bulk copies are bounded too:
+    ``lost_draw_request`` makes it skip the first staging of one request's
+    draw, that wait runs out, and the request reports -2."""
+    w = make_workload(B=12, k_max=4, V=V, dtype=dtype, seed=73, boost=3.0, draft_noise=0.5, draft_mode=mode,
+                      lens=[4, 3, 4, 2, 4, 4, 1, 4, 0, 4, 3, 4])
+    d = device_inputs(w, misalign=misalign)
+    kernel = sv.StatsKernel.SCALAR if misalign else TMA
+
+    def run(**kw):
+        n, t = sv.spec_verify(d["target"], d["draft"], d["tokens"], d["lens"], d["uniforms"], w.temperature,
+                              V=w.V, stats_kernel=kernel, **kw)
+        torch.cuda.synchronize()
+        return n.cpu().numpy(), t.cpu().numpy()
+
+    clean = run()
+    assert np.all(clean[0] >= 0)
+    victims = draw_victims(clean[0], w)
+    assert victims
+    for victim in victims:
+        n, t = run(wait_timeout_us=20000, lost_draw_request=victim + 1)
+        assert n[victim] == -2 and np.all(t[victim] == -1)
+        lost = n == -2
+        assert np.all(t[lost] == -1)
+        assert np.array_equal(n[~lost], clean[0][~lost]) and np.array_equal(t[~lost], clean[1][~lost])
+        assert lost.sum() < w.B
+        again = run()
+        assert np.array_equal(again[0], clean[0]) and np.array_equal(again[1], clean[1])
