@@ -543,6 +543,93 @@ def pin_accept_sim_matches_verify_and_monte_carlo(orc):
     assert abs(np.mean(js) - e) < 5 * sd + 1e-9, (np.mean(js), e, sd)
 
 
+# --------------------------------------------------------------------------
+# Near-tie flags (the benchmark spec: the generator and oracle flag positions where
+# |u - min(1, p/q)| or the residual-CDF margin is below 1e-5) and the two
+# fallback branches of the rule's readings (no step above u*W: the largest
+# positive-weight token; zero residual mass: draw from p_j).
+
+
+def _flags(orc, target, draft, tokens, u, T=1.0):
+    j, toks, flags = run1(orc, target, draft, tokens, u, T)
+    return j, toks, flags
+
+
+def pin_accept_tie_band(orc):
+    from oracle import FLAG_ACCEPT_TIE
+    # a = p(x) = 0.3 for a one-hot draft; a = p/q = 0.3/0.6 = 0.5 with a draft row
+    target = [[math.log(0.3), math.log(0.7)], [0.0, 0.0]]
+    cases = [(None, 0.3), ([[math.log(0.6), math.log(0.4)]], 0.5)]
+    for draft, a in cases:
+        for du, flagged in ((5e-6, True), (-5e-6, True), (2e-5, False), (-2e-5, False), (0.3, False)):
+            u0 = a + du
+            if not 0.0 <= u0 < 1.0:
+                continue
+            j, _, flags = _flags(orc, target, draft, [0], [u0, 0.5])
+            assert bool(flags & FLAG_ACCEPT_TIE) == flagged, (a, du, flags)
+            assert j == (1 if u0 < a else 0), (a, du, j)
+    # a tie after the first rejection is never examined, so it is not flagged
+    target3 = [[math.log(0.3), math.log(0.7)]] * 3
+    j, _, flags = _flags(orc, target3, None, [0, 0], [0.9, 0.3, 0.5])
+    assert j == 0 and not flags & FLAG_ACCEPT_TIE, (j, flags)
+
+
+def pin_draw_tie_band(orc):
+    from oracle import FLAG_DRAW_TIE
+    # bonus draw (k = 0) from p = [1/4, 1/2, 1/4]: CDF steps at 0.25 and 0.75, W = 1
+    row = np.log(np.array([1.0, 2.0, 1.0]) / 4.0).astype(np.float32)
+    for step, below, above in ((0.25, 0, 1), (0.75, 1, 2)):
+        for du, flagged in ((0.5e-5, True), (-0.5e-5, True), (2e-5, False), (-2e-5, False)):
+            out = orc.verify(row[None, None], None, np.zeros((1, 0), np.int32), None,
+                             np.array([[step + du]]), 1.0)
+            flags, tok = int(out["flags"][0]), int(out["tokens"][0, 0])
+            assert bool(flags & FLAG_DRAW_TIE) == flagged, (step, du, flags)
+            assert tok == (above if du > 0 else below), (step, du, tok)
+    # the band is relative to W: a one-hot rejection at x = 1 leaves the
+    # residual [1/4, 0, 1/4] (W = 1/2, step at 1/4 in weight, u* = 1/2 there);
+    # u* off by 1.5e-5 puts u*W 0.75e-5 from the step: inside an absolute
+    # 1e-5 band, outside the relative one (1e-5 W = 0.5e-5)
+    target = np.stack([row, row])
+    for du, flagged in ((0.5e-5, True), (-0.5e-5, True), (1.5e-5, False), (-1.5e-5, False)):
+        j, toks, flags = _flags(orc, target, None, [1], [0.9, 0.5 + du])
+        assert j == 0 and toks[0] == (2 if du > 0 else 0), (du, j, toks)
+        assert bool(flags & FLAG_DRAW_TIE) == flagged, (du, flags)
+
+
+def pin_draw_fallback_takes_last_positive_weight(orc):
+    from oracle import FLAG_DRAW_FALLBACK
+    # p = [1/2, 1/2, 0, 0]; u* = 1 leaves no token t with C_t > u* W, so the
+    # rule's fallback applies: the largest t with positive weight (1, not the
+    # last index 3 and not the first positive index 0)
+    row = np.array([0.0, 0.0, -np.inf, -np.inf], np.float32)
+    out = orc.verify(row[None, None], None, np.zeros((1, 0), np.int32), None, np.array([[1.0]]), 1.0)
+    assert int(out["tokens"][0, 0]) == 1, out["tokens"]
+    assert int(out["flags"][0]) & FLAG_DRAW_FALLBACK
+    # away from it the ordinary rule holds and the fallback flag stays clear
+    out = orc.verify(row[None, None], None, np.zeros((1, 0), np.int32), None, np.array([[0.25]]), 1.0)
+    assert int(out["tokens"][0, 0]) == 0 and not int(out["flags"][0]) & FLAG_DRAW_FALLBACK
+
+
+def pin_zero_residual_draws_from_p(orc):
+    from oracle import FLAG_ZERO_RESIDUAL
+    # identical draft: p == q, so a = 1; u_0 = 1 (no uniform in [0, 1) can do
+    # it) forces the rejection, the residual max(0, p - q) is all zero, and
+    # the draw falls back to p_0 = [1/4, 1/2, 1/4]
+    row = np.log(np.array([1.0, 2.0, 1.0]) / 4.0).astype(np.float32)
+    target = np.stack([row, row])
+    for us, want in ((0.1, 0), (0.6, 1), (0.9, 2)):
+        j, toks, flags = _flags(orc, target, row[None], [1], [1.0, us])
+        assert j == 0 and toks[0] == want, (us, j, toks)
+        assert flags & FLAG_ZERO_RESIDUAL
+        # one-hot draft at a token with p = 1: the residual is zero as well
+    certain = np.array([[0.0, -np.inf], [0.0, 0.0]], np.float32)
+    j, toks, flags = _flags(orc, certain, None, [0], [1.0, 0.7])
+    assert j == 0 and toks[0] == 0 and flags & FLAG_ZERO_RESIDUAL, (j, toks, flags)
+    # an ordinary rejection never sets the flag
+    j, toks, flags = _flags(orc, target, None, [1], [0.9, 0.6])
+    assert j == 0 and not flags & FLAG_ZERO_RESIDUAL
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_lse_closed_forms,
@@ -555,6 +642,10 @@ ALL_PINS = [
     pin_never_draws_zero_weight,
     pin_inverse_cdf_matches_searchsorted,
     pin_lens_zero,
+    pin_accept_tie_band,
+    pin_draw_tie_band,
+    pin_draw_fallback_takes_last_positive_weight,
+    pin_zero_residual_draws_from_p,
     pin_lossless_enumeration,
     pin_lossless_chi_square,
     pin_sequential_rule,

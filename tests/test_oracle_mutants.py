@@ -58,6 +58,24 @@ MUTANTS = [
      "(i <= j ? 1.0 : pow(decay, (double)(i - j)))", "pow(decay, (double)i)"),
     ("acceptance probability not clamped at one",
      "                a[i] = r > 1.0 ? 1.0 : r;", "                a[i] = r;"),
+    ("acceptance tie band 1e-3",
+     "if (fabs(u[i] - a) < ORACLE_TIE_BAND)", "if (fabs(u[i] - a) < 1e-3)"),
+    ("acceptance tie band 1e-7",
+     "if (fabs(u[i] - a) < ORACLE_TIE_BAND)", "if (fabs(u[i] - a) < 1e-7)"),
+    ("draw tie band 1e-3 of W",
+     "fabs(C - target) < ORACLE_TIE_BAND * W)", "fabs(C - target) < 1e-3 * W)"),
+    ("draw tie band 1e-7 of W",
+     "            if (fabs(target - C_prev) < ORACLE_TIE_BAND * W ||\n                fabs(C - target) < ORACLE_TIE_BAND * W)",
+     "            if (fabs(target - C_prev) < 1e-7 * W ||\n                fabs(C - target) < 1e-7 * W)"),
+    ("draw tie band absolute instead of relative to W",
+     "            if (fabs(target - C_prev) < ORACLE_TIE_BAND * W ||\n                fabs(C - target) < ORACLE_TIE_BAND * W)",
+     "            if (fabs(target - C_prev) < ORACLE_TIE_BAND ||\n                fabs(C - target) < ORACLE_TIE_BAND)"),
+    ("fallback takes the first positive weight",
+     "    for (int64_t t = V - 1; t >= 0; --t)\n        if (w[t] > 0.0)",
+     "    for (int64_t t = 0; t < V; ++t)\n        if (w[t] > 0.0)"),
+    ("zero residual mass keeps the zero weights",
+     "            for (int64_t v = 0; v < V; ++v)\n                w[v] = exp(ell_t[v] - lse_t_row[j]);\n        }",
+     "        }"),
 ]
 
 
