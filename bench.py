@@ -493,14 +493,32 @@ def main():
 
 class DeviceWorkload:
     """One workload resident on the device, with its output buffers and
-    workspace, and the call that verifies it."""
+    workspace, and the call that verifies it.
+
+    Workloads smaller than twice the L2 cache are held in N device copies and
+    step i verifies copy i mod N, with N chosen so that at least 2 x L2 of
+    other inputs are read between two uses of one copy: every step reads its
+    logits from HBM, as a fresh batch would be, and no cache flush (whose
+    dirty lines would be written back inside the timed step) is needed."""
 
     def __init__(self, sv, torch, dev, stream, w, greedy, kernel):
         self.sv, self.torch, self.dev, self.stream, self.w = sv, torch, dev, stream, w
         self.greedy, self.kernel = greedy, kernel
         self.is_bf16 = w.dtype == "bf16"
-        t = lambda a, bf=False: (torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16) if bf
-                                 else torch.from_numpy(np.ascontiguousarray(a))).to(dev)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.in_bytes = input_bytes(w, greedy)
+        self.copies = 1 if self.in_bytes >= 2 * l2 else -(-2 * l2 // self.in_bytes) + 1
+
+        def t(a, bf=False):
+            x = torch.from_numpy(np.ascontiguousarray(a))
+            if bf:
+                x = x.view(torch.bfloat16)
+            x = x.to(dev)
+            if self.copies == 1:
+                return [x]
+            stacked = x.unsqueeze(0).repeat(self.copies, *([1] * x.dim())).contiguous()
+            return [stacked[i] for i in range(self.copies)]
+
         self.target = t(w.target, self.is_bf16)
         self.draft = None if (w.draft is None or greedy) else t(w.draft, self.is_bf16)
         self.tokens = t(w.tokens)
@@ -510,21 +528,22 @@ class DeviceWorkload:
                     torch.empty(w.B, w.k_max + 1, dtype=torch.int32, device=dev))
         self.ws = torch.empty(max(sv.workspace_bytes(w.B, w.k_max, w.V, sv.BF16 if self.is_bf16 else sv.F32), 256),
                               dtype=torch.uint8, device=dev)
-        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-        self.in_bytes = input_bytes(w, greedy)
-        self.flush_buf = None
-        if self.in_bytes < 2 * l2:
-            self.flush_buf = torch.empty(4 * l2 // 4, dtype=torch.int32, device=dev)
         self.l2_note = (f"inputs {self.in_bytes / 1e6:.1f} MB > 2 x L2 ({l2 / 2**20:.0f} MiB): no flush"
-                        if self.flush_buf is None else
-                        f"inputs {self.in_bytes / 1e6:.1f} MB < 2 x L2: L2 flushed (write "
-                        f"{self.flush_buf.numel() * 4 / 2**20:.0f} MiB) before every step, outside each step's events")
+                        if self.copies == 1 else
+                        f"inputs {self.in_bytes / 1e6:.1f} MB < 2 x L2 ({l2 / 2**20:.0f} MiB): {self.copies} device "
+                        f"copies, step i reads copy i mod {self.copies} "
+                        f"({(self.copies - 1) * self.in_bytes / 1e6:.0f} MB of other inputs between two reads of one "
+                        f"copy), no flush")
+        self._i = 0
 
-    def step(self, events=None):
+    def step(self, events=None, copy=None):
         w = self.w
-        self.sv.spec_verify(self.target, self.draft, self.tokens, self.lens, self.uniforms, w.temperature,
-                            self.greedy, V=w.V, out=self.out, workspace=self.ws, stream=self.stream,
-                            stats_kernel=self.kernel, events=events)
+        c = self._i % self.copies if copy is None else copy
+        self._i += 1
+        pick = lambda x: None if x is None else x[c]
+        self.sv.spec_verify(pick(self.target), pick(self.draft), pick(self.tokens), pick(self.lens),
+                            pick(self.uniforms), w.temperature, self.greedy, V=w.V, out=self.out, workspace=self.ws,
+                            stream=self.stream, stats_kernel=self.kernel, events=events)
 
     def event(self):
         e = self.torch.cuda.Event(enable_timing=True)
@@ -532,37 +551,21 @@ class DeviceWorkload:
         return e
 
     def time_steps(self, steps, warmup, barrier=lambda: None):
-        """Time `steps` calls; returns (device ms over the timed calls,
-        region ms).  Without an L2 flush the calls run back to back between
-        two events; with one, every call is bracketed by its own events and
-        the flush stays outside them."""
+        """Time `steps` calls back to back between two events; returns the
+        device ms of the timed calls."""
         torch = self.torch
         for _ in range(warmup):
             self.step()
         torch.cuda.synchronize()
-        step_ev = [(None, None)] * steps
-        g0 = g1 = None
         barrier()
         torch.cuda.synchronize()
-        if self.flush_buf is None:
-            g0 = self.event()
-            for _ in range(steps):
-                self.step()
-            g1 = self.event()
-        else:
-            step_ev = []
-            for i in range(steps):
-                self.flush_buf.fill_(i)
-                a = self.event()
-                self.step()
-                step_ev.append((a, self.event()))
+        g0 = self.event()
+        for _ in range(steps):
+            self.step()
+        g1 = self.event()
         torch.cuda.synchronize()
         barrier()
-        if self.flush_buf is None:
-            region = g0.elapsed_time(g1)
-            return region, region
-        per = [a.elapsed_time(b) for a, b in step_ev]
-        return sum(per), sum(per)
+        return g0.elapsed_time(g1)
 
     def time_k1(self, samples):
         """The row-statistics kernel alone: `samples` calls, each with events
@@ -571,9 +574,7 @@ class DeviceWorkload:
         Returns the per-launch times in ms."""
         torch = self.torch
         ev = []
-        for i in range(samples):
-            if self.flush_buf is not None:
-                self.flush_buf.fill_(i)
+        for _ in range(samples):
             # recorded once here so that torch creates the events; the
             # library records them again around the row-statistics kernel
             a, b = self.event(), self.event()
@@ -588,7 +589,7 @@ class DeviceWorkload:
         token is a vocabulary id and -1 fills the rest; and the host entry
         point (spec_verify_host, host buffers) returns the same outputs."""
         torch, w = self.torch, self.w
-        self.step()
+        self.step(copy=0)
         torch.cuda.synchronize()
         g_len = self.out[0].cpu().numpy()
         g_tok = self.out[1].cpu().numpy()
@@ -623,7 +624,7 @@ class DeviceWorkload:
         return self._host
 
     def release(self):
-        for name in ("target", "draft", "tokens", "lens", "uniforms", "out", "ws", "flush_buf", "_host"):
+        for name in ("target", "draft", "tokens", "lens", "uniforms", "out", "ws", "_host"):
             setattr(self, name, None)
 
 
@@ -640,14 +641,14 @@ def reread_bytes(w, g_len, greedy=False) -> int:
 def launches_per_call(B: int, greedy: bool) -> int:
     """Kernels one spec_verify call launches: the row-statistics kernel per
     block of up to 4096 requests, the scan kernel, and (sampling) the draw
-    kernel."""
-    return math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + 1 + (0 if greedy else 1)
+    and selection kernels."""
+    return math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + 1 + (0 if greedy else 2)
 
 
 def config_record(dw, cfg, steps, warmup, k1_samples, peak):
     """Per-workload figures for the per_config block of the bench line."""
     w = dw.w
-    dev_ms, _ = dw.time_steps(steps, warmup)
+    dev_ms = dw.time_steps(steps, warmup)
     k1 = dw.time_k1(k1_samples)
     g_len, parity = dw.host_check()
     alg = stats_pass_bytes(w, dw.greedy)
@@ -701,7 +702,8 @@ def run_ours_impl(args):
 
     K, W = args.steps, args.warmup
     with ClockSampler(local_rank) as clocks:
-        t_rank, region_ms = dw.time_steps(K, W, barrier)
+        t_rank = dw.time_steps(K, W, barrier)
+    region_ms = t_rank
     t_max = max_over_ranks(t_rank, dev)
     positions = w.positions
     value = aggregate_value(n, positions, K, t_max)

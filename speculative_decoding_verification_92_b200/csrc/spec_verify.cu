@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "spec_verify.h"
 #include "sv_common.cuh"
@@ -21,6 +22,11 @@ namespace {
 constexpr int kTmaConsumerWarps = SV_TMA_CONSUMER_WARPS;
 constexpr int kTmaStages = SV_TMA_STAGES;
 constexpr int kLdgThreads = 256;
+// Share of the pieces the bulk-copy row-statistics kernel splits statically
+// (the rest is handed out piece by piece).
+#ifndef SV_STATIC_PCT
+#define SV_STATIC_PCT 50
+#endif
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 
@@ -147,10 +153,18 @@ bool shape_ok(const sv_shape* s, sv_status* why) {
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Workspace: the row-statistics partials, then the draw queue the scan
-// kernel fills and the draw kernel drains.
+// Control words, zeroed (cudaMemsetAsync) before every call: [0] residual
+// draws queued, [1] one-piece draws queued, [2 + l] the pieces the l-th
+// row-statistics launch (up to 4096 requests each) has handed out.
+int64_t stats_launches(const sv_shape& s) {
+    return (int64_t(s.B) + kMaxRequestsPerLaunch - 1) / kMaxRequestsPerLaunch;
+}
+int64_t ctrl_ints(const sv_shape& s) { return 2 + stats_launches(s); }
+
+// Workspace: the row-statistics partials, the control words, then the draw
+// queue the scan kernel fills and the draw kernel drains.
 struct WsLayout {
-    size_t partials, ctrl, res_req, one_req, res_cnt, seg, total;
+    size_t partials, ctrl, res_req, one_req, res_lost, seg, total;
 };
 
 WsLayout ws_layout(const sv_shape& s, const Plan& p) {
@@ -158,10 +172,10 @@ WsLayout ws_layout(const sv_shape& s, const Plan& p) {
     WsLayout l{};
     size_t off = 0;
     l.partials = off; off += align256(B * size_t(2 * s.k_max + 1) * size_t(p.P) * sizeof(float2));
-    l.ctrl = off;     off += 256;
+    l.ctrl = off;     off += align256(ctrl_ints(s) * sizeof(int32_t));
     l.res_req = off;  off += align256(B * sizeof(DrawReq));
     l.one_req = off;  off += align256(B * sizeof(DrawReq));
-    l.res_cnt = off;  off += align256(B * sizeof(int32_t));
+    l.res_lost = off; off += align256(B * sizeof(int32_t));
     l.seg = off;      off += align256(B * size_t(p.P) * kSegsPerPiece * sizeof(float));
     l.total = off;
     return l;
@@ -171,11 +185,19 @@ size_t workspace_bytes_for(const sv_shape& s, const Plan& p) { return ws_layout(
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
+// NVTX range around the launches of one kernel (header-only NVTX: a no-op
+// unless a profiler is attached), so timelines name the phases of a call.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+
 template <typename T, bool kGreedy>
 cudaError_t launch_stats(const StatsParams& base, int B, int variant, const DeviceInfo& dev, cudaStream_t st) {
     for (int b0 = 0; b0 < B; b0 += kMaxRequestsPerLaunch) {
         StatsParams prm = base;
         prm.b0 = b0;
+        prm.dyn_ticket = base.dyn_ticket + b0 / kMaxRequestsPerLaunch;
         prm.nB = B - b0 < kMaxRequestsPerLaunch ? B - b0 : kMaxRequestsPerLaunch;
         const int rows_max = prm.use_draft ? 2 * prm.k_max + 1 : prm.k_max + 1;
         const int64_t items_upper = int64_t(prm.nB) * rows_max * prm.P;
@@ -223,48 +245,53 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
     return cudaSuccess;
 }
 
-// K2a, one CTA per request, then K2b (sampling), each a programmatic
-// dependent of the kernel before it.
+// K2a (one CTA per request), then for sampling K2b (persistent, one wave) and
+// K2c (one warp per possible residual draw), each a programmatic dependent of
+// the kernel before it.
 template <typename T>
-cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, int B, bool draw, const DeviceInfo& dev,
-                             cudaStream_t st) {
+cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, const SelectParams& cp, int B, bool draw,
+                             const DeviceInfo& dev, cudaStream_t st) {
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    {
-        auto k = verify_scan_kernel<T>;
-        const size_t smem = scan_smem_bytes(sp.k_max);
-        cudaError_t e = allow_smem(k, smem);
-        if (e != cudaSuccess) return e;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(B));
-        cfg.blockDim = dim3(kScanThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if ((e = cudaLaunchKernelEx(&cfg, k, sp)) != cudaSuccess) return e;
-    }
-    if (!draw) return cudaSuccess;
-    auto k = verify_draw_kernel<T>;
-    cudaError_t e = allow_smem(k, kDrawSmemBytes);
-    if (e != cudaSuccess) return e;
-    // persistent: at most one wave of resident CTAs, and no more than the
-    // largest possible number of tasks
-    int per_sm = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kDrawThreads, kDrawSmemBytes)) != cudaSuccess)
-        return e;
-    per_sm = per_sm < 1 ? 1 : (per_sm > kDrawCtasPerSm ? kDrawCtasPerSm : per_sm);
-    const int64_t cap = int64_t(dev.sm_count) * per_sm;
-    const int64_t max_tasks = int64_t(B) * (dp.P + 1);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(max_tasks < cap ? max_tasks : cap));
-    cfg.blockDim = dim3(kDrawThreads);
-    cfg.dynamicSmemBytes = kDrawSmemBytes;
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k, dp);
+    {
+        auto k = verify_scan_kernel<T>;
+        const size_t smem = scan_smem_bytes(sp.k_max, sp.P);
+        cudaError_t e = allow_smem(k, smem);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3(static_cast<unsigned>(B));
+        cfg.blockDim = dim3(kScanThreads);
+        cfg.dynamicSmemBytes = smem;
+        if ((e = cudaLaunchKernelEx(&cfg, k, sp)) != cudaSuccess) return e;
+    }
+    if (!draw) return cudaSuccess;
+    {
+        auto k = verify_draw_kernel<T>;
+        cudaError_t e = allow_smem(k, kDrawSmemBytes);
+        if (e != cudaSuccess) return e;
+        // persistent: at most one wave of resident CTAs, and no more than the
+        // largest possible number of tasks
+        int per_sm = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kDrawThreads, kDrawSmemBytes)) !=
+            cudaSuccess)
+            return e;
+        per_sm = per_sm < 1 ? 1 : (per_sm > kDrawCtasPerSm ? kDrawCtasPerSm : per_sm);
+        const int64_t cap = int64_t(dev.sm_count) * per_sm;
+        const int64_t max_tasks = int64_t(B) * (dp.P + 1);
+        cfg.gridDim = dim3(static_cast<unsigned>(max_tasks < cap ? max_tasks : cap));
+        cfg.blockDim = dim3(kDrawThreads);
+        cfg.dynamicSmemBytes = kDrawSmemBytes;
+        if ((e = cudaLaunchKernelEx(&cfg, k, dp)) != cudaSuccess) return e;
+    }
+    auto k = verify_select_kernel<T>;
+    cfg.gridDim = dim3(static_cast<unsigned>((int64_t(B) + kSelectWarps - 1) / kSelectWarps));
+    cfg.blockDim = dim3(kSelectThreads);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, k, cp);
 }
 
 struct Call {
@@ -303,42 +330,15 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     const WsLayout wl = ws_layout(s, plan);
     unsigned char* ws = static_cast<unsigned char*>(a.workspace);
     int32_t* ctrl = reinterpret_cast<int32_t*>(ws + wl.ctrl);
-    StatsParams sp{};
-    sp.target = static_cast<const unsigned char*>(a.target);
-    sp.draft = static_cast<const unsigned char*>(a.draft);
-    sp.lens = a.lens;
-    sp.partials = reinterpret_cast<float2*>(ws + wl.partials);
-    sp.ctrl = ctrl;
-    sp.k_max = s.k_max;
-    sp.V = s.V;
-    sp.row_stride = plan.stride;
-    sp.P = plan.P;
-    sp.PE = plan.PE;
-    sp.scale = greedy ? 1.f : static_cast<float>(kLog2e / static_cast<double>(a.temperature));
-    sp.use_draft = (a.draft != nullptr && !greedy) ? 1 : 0;
-    const int tmo = a.opts ? a.opts->wait_timeout_us : 0;
-    sp.timeout_ns = tmo > 0 ? uint64_t(tmo) * 1000ull : kDefaultTimeoutNs;
-    const int lost = a.opts ? a.opts->lost_copy_request : 0;
-    sp.lost_copy_partial = lost > 0 ? int64_t(lost - 1) * (2 * s.k_max + 1) * plan.P : -1;
-
-    cudaError_t e = cudaSuccess;
-    if (a.opts && a.opts->event_stats_begin)
-        if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_begin), a.stream)) != cudaSuccess)
-            return SV_ECUDA;
-    e = greedy ? launch_stats<T, true>(sp, s.B, variant, dev, a.stream)
-               : launch_stats<T, false>(sp, s.B, variant, dev, a.stream);
-    if (e != cudaSuccess) return SV_ECUDA;
-    if (a.opts && a.opts->event_stats_end)
-        if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_end), a.stream)) != cudaSuccess)
-            return SV_ECUDA;
+    const float scale = greedy ? 1.f : static_cast<float>(kLog2e / static_cast<double>(a.temperature));
 
     ScanParams cp{};
-    cp.target = sp.target;
-    cp.draft = greedy ? nullptr : sp.draft;
+    cp.target = static_cast<const unsigned char*>(a.target);
+    cp.draft = greedy ? nullptr : static_cast<const unsigned char*>(a.draft);
     cp.tokens = a.tokens;
     cp.lens = a.lens;
     cp.uniforms = a.uniforms;
-    cp.partials = sp.partials;
+    cp.partials = reinterpret_cast<float2*>(ws + wl.partials);
     cp.out_len = a.out_len;
     cp.out_tokens = a.out_tokens;
     cp.out_lse_t = a.out_lse_t;
@@ -353,24 +353,59 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     cp.ctrl = ctrl;
     cp.res_req = reinterpret_cast<DrawReq*>(ws + wl.res_req);
     cp.one_req = reinterpret_cast<DrawReq*>(ws + wl.one_req);
-    cp.res_cnt = reinterpret_cast<int32_t*>(ws + wl.res_cnt);
+    cp.res_lost = reinterpret_cast<int32_t*>(ws + wl.res_lost);
     cp.k_max = s.k_max;
     cp.V = s.V;
     cp.row_stride = plan.stride;
     cp.P = plan.P;
     cp.PE = plan.PE;
-    cp.scale = sp.scale;
+    cp.scale = scale;
     cp.greedy = greedy ? 1 : 0;
     cp.stats_only = a.stats_only ? 1 : 0;
 
+    StatsParams sp{};
+    sp.target = static_cast<const unsigned char*>(a.target);
+    sp.draft = static_cast<const unsigned char*>(a.draft);
+    sp.lens = a.lens;
+    sp.partials = reinterpret_cast<float2*>(ws + wl.partials);
+    sp.dyn_ticket = ctrl + 2;
+    sp.static_pct = SV_STATIC_PCT;
+    sp.k_max = s.k_max;
+    sp.V = s.V;
+    sp.row_stride = plan.stride;
+    sp.P = plan.P;
+    sp.PE = plan.PE;
+    sp.scale = scale;
+    sp.use_draft = (a.draft != nullptr && !greedy) ? 1 : 0;
+    const int tmo = a.opts ? a.opts->wait_timeout_us : 0;
+    sp.timeout_ns = tmo > 0 ? uint64_t(tmo) * 1000ull : kDefaultTimeoutNs;
+    const int lost = a.opts ? a.opts->lost_copy_request : 0;
+    sp.lost_copy_partial = lost > 0 ? int64_t(lost - 1) * (2 * s.k_max + 1) * plan.P : -1;
+
+    cudaError_t e = cudaMemsetAsync(ctrl, 0, size_t(ctrl_ints(s)) * sizeof(int32_t), a.stream);
+    if (e != cudaSuccess) return SV_ECUDA;
+    if (a.opts && a.opts->event_stats_begin)
+        if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_begin), a.stream)) != cudaSuccess)
+            return SV_ECUDA;
+    {
+        NvtxRange range("spec_verify: row statistics");
+        e = greedy ? launch_stats<T, true>(sp, s.B, variant, dev, a.stream)
+                   : launch_stats<T, false>(sp, s.B, variant, dev, a.stream);
+    }
+    if (e != cudaSuccess) return SV_ECUDA;
+    if (a.opts && a.opts->event_stats_end)
+        if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_end), a.stream)) != cudaSuccess)
+            return SV_ECUDA;
+
     DrawParams dp{};
+    dp.B = s.B;
     dp.target = sp.target;
     dp.draft = cp.draft;
     dp.partials = sp.partials;
     dp.ctrl = ctrl;
     dp.res_req = cp.res_req;
     dp.one_req = cp.one_req;
-    dp.res_cnt = cp.res_cnt;
+    dp.res_lost = cp.res_lost;
     dp.seg = reinterpret_cast<float*>(ws + wl.seg);
     dp.out_len = a.out_len;
     dp.out_tokens = a.out_tokens;
@@ -379,12 +414,33 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     dp.row_stride = plan.stride;
     dp.P = plan.P;
     dp.PE = plan.PE;
-    dp.scale = sp.scale;
+    dp.scale = scale;
     dp.rows_aligned = rows_aligned ? 1 : 0;
     dp.timeout_ns = sp.timeout_ns;
     const int lost_draw = a.opts ? a.opts->lost_draw_request : 0;
     dp.lost_draw_b = lost_draw > 0 ? lost_draw - 1 : -1;
-    e = launch_scan_draw<T>(cp, dp, s.B, !greedy && !a.stats_only, dev, a.stream);
+    SelectParams xp{};
+    xp.B = s.B;
+    xp.target = dp.target;
+    xp.draft = dp.draft;
+    xp.partials = dp.partials;
+    xp.ctrl = ctrl;
+    xp.res_req = dp.res_req;
+    xp.seg = dp.seg;
+    xp.res_lost = dp.res_lost;
+    xp.out_len = a.out_len;
+    xp.out_tokens = a.out_tokens;
+    xp.k_max = s.k_max;
+    xp.V = s.V;
+    xp.row_stride = plan.stride;
+    xp.P = plan.P;
+    xp.PE = plan.PE;
+    xp.scale = scale;
+    xp.rows_aligned = dp.rows_aligned;
+    {
+        NvtxRange range("spec_verify: scan, draw, selection");
+        e = launch_scan_draw<T>(cp, dp, xp, s.B, !greedy && !a.stats_only, dev, a.stream);
+    }
     return e == cudaSuccess ? SV_OK : SV_ECUDA;
 }
 

@@ -146,6 +146,25 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
         : "memory");
 }
 
+// L2 policy for data read once: its lines are the first to be evicted, so a
+// stream of logits does not push out what later kernels read again (their
+// code, the row-statistics partials, the draw queue).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// bulk_copy_g2s with an L2 cache policy (l2_evict_first_policy).
+__device__ __forceinline__ void bulk_copy_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                                   uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared memory (L2 only), grouped with
 // cp_async_commit and awaited with cp_async_wait<N> (at most N newest groups
 // still pending).  Both addresses must be 16-byte aligned.

@@ -2,9 +2,13 @@
 //
 // Every row a request uses (target rows 0..L_b, draft rows 0..L_b-1) is cut
 // into P pieces of PE elements (16 KiB each, the last one ragged).  The
-// pieces of all used rows, in request order, form one list; CTA x of a grid
-// of G takes the contiguous range [x*N/G, (x+1)*N/G) of the N pieces, so
-// every CTA streams the same number of bytes give or take one piece.  Each
+// pieces of all used rows, in request order, form one list of N pieces.
+// Bulk-copy variant: CTA x of a grid of G first takes the contiguous range
+// [x*S, (x+1)*S) with S = floor(N * static_pct / 100 / G), then pieces
+// G*S, G*S + 1, ... one at a time from a shared counter, so CTAs that stream
+// faster (SMs do not all get the same share of HBM bandwidth) take more
+// pieces and all CTAs finish within about one piece of each other.  The
+// element-load variant takes the contiguous range [x*N/G, (x+1)*N/G).  Each
 // piece is reduced to one partial:
 //   sampling: (m, s) with m = max_v t_v, s = sum_v 2^(t_v - m), t_v = z_v * log2(e)/T
 //             (the temperature softmax statistics of step 1 of the rule,
@@ -63,8 +67,8 @@ struct StatsParams {
     const unsigned char* draft;   // [B][k_max][row_stride] or null
     const int32_t* lens;          // [B] or null (all k_max)
     float2* partials;             // [B][2*k_max+1][P]
-    int32_t* ctrl;                // the draw kernels' list counters: zeroed by block 0 of the
-                                  // launch with b0 == 0 (null: nothing to zero)
+    int32_t* dyn_ticket;          // this launch's counter of handed-out pieces (zero at launch; the
+                                  // bulk-copy variant only)
     int32_t b0;                   // first request handled by this launch
     int32_t nB;                   // requests handled by this launch (<= kMaxRequestsPerLaunch)
     int32_t k_max;
@@ -76,6 +80,7 @@ struct StatsParams {
     int32_t use_draft;            // draft rows are part of the work
     uint64_t timeout_ns;          // bound on each barrier wait (TMA variant)
     int64_t lost_copy_partial;    // test fault injection: this piece is never copied; -1 = off
+    int32_t static_pct;           // bulk-copy variant: percent of the pieces split statically
 };
 
 struct ItemDesc {
@@ -393,13 +398,6 @@ __device__ __forceinline__ void fold_vector(Acc<kGreedy>& acc, const uint4& w, i
     }
 }
 
-__device__ __forceinline__ void zero_ctrl(const StatsParams& p) {
-    if (p.ctrl && p.b0 == 0 && blockIdx.x == 0 && threadIdx.x == 0) {
-        p.ctrl[0] = 0;
-        p.ctrl[1] = 0;
-    }
-}
-
 // ============================================================================
 // TMA bulk-copy variant.
 
@@ -412,7 +410,7 @@ struct StageMeta {
     const unsigned char* tail;  // first ragged-tail element (row's last piece), or null
     int64_t partial_idx;
     int32_t elem0;              // row index of the stage's first element
-    int32_t n_bytes;            // bytes delivered by the bulk copy (multiple of 16)
+    int32_t n_bytes;            // bytes delivered by the bulk copy (multiple of 16); -1: no more pieces
     int32_t tail_n;             // ragged-tail elements (< 16 / sizeof element)
     int32_t pad;
 };
@@ -423,7 +421,7 @@ struct TmaSmem {
     static constexpr size_t kBarOff = kMetaOff + sizeof(StageMeta) * kStages;
     static constexpr size_t kMiscOff = kBarOff + 16 * kStages;                         // full[], empty[]
     static constexpr size_t kPartOff = kMiscOff + 4 * 64;                              // misc ints
-    static constexpr size_t kRowOff = kPartOff + 8 * size_t(kStages) * kConsumerWarps * 32;  // part[stage][thread]
+    static constexpr size_t kRowOff = kPartOff + 8 * size_t(2 * kStages) * kConsumerWarps * 32;  // part[round&1][stage][thread]
     static size_t bytes(int nB) { return kRowOff + 4 * size_t(nB + 1); }
 };
 
@@ -455,11 +453,14 @@ row_stats_tma_kernel(const StatsParams p) {
     uint64_t* empty = full + kStages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff);
     int* scan_scratch = reinterpret_cast<int*>(smem + L::kMiscOff) + 8;
-    float2* part = reinterpret_cast<float2*>(smem + L::kPartOff);   // [kStages][kConsumers]
+    float2* part = reinterpret_cast<float2*>(smem + L::kPartOff);   // [2][kStages][kConsumers]
     int* row_start = reinterpret_cast<int*>(smem + L::kRowOff);
 
     const int tid = threadIdx.x;
-    zero_ctrl(p);
+    // The scan kernel may be launched now: its CTAs take the places of this
+    // grid's CTAs as they exit (this grid is one resident wave) and run their
+    // input-only prologue, then wait for this grid to complete.
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full + s, 1);
@@ -469,64 +470,114 @@ row_stats_tma_kernel(const StatsParams p) {
         fence_mbar_init();
     }
     build_row_prefix<kThreads>(p, row_start, scan_scratch);  // ends with __syncthreads
-    int64_t lo, hi;
-    piece_range((int64_t)row_start[p.nB] * p.P, &lo, &hi);
+    const int64_t total = (int64_t)row_start[p.nB] * p.P;
 
     if (tid >= kConsumers) {
         // ----------------------------- producer warp -----------------------------
-        // Issues piece `next` into stage (next - lo) % kStages while the ring
-        // has room; otherwise waits until the consumers have released the
-        // oldest piece in flight, merges their per-thread partials of it and
-        // stores the piece's partial.  Stage s receives its r-th piece in
-        // round r; the consumers' release of it is the r-th completion of
-        // empty[s] (parity r & 1), the copy's arrival the r-th of full[s].
+        // The i-th item issued goes to stage i % kStages in round i / kStages:
+        // the copy's arrival is that round's completion of full[stage], the
+        // consumers' release of it the same round's completion of empty[stage]
+        // (parity round & 1).  After the last piece the producer posts an end
+        // marker (no copy) that stops the consumers.  While the ring is full
+        // it waits for the oldest piece's release, refills that stage at once
+        // and only then merges the consumers' per-thread partials of the
+        // released piece (they live in part[round & 1][stage], so the
+        // consumers of the next round never overwrite them before the merge).
         const int lane = tid - kConsumers;
-        int64_t next = lo, merged = lo;
+        const uint64_t stream_policy = l2_evict_first_policy();  // logits are read once
+        const int64_t S = total * p.static_pct / 100 / gridDim.x;  // static pieces per CTA
+        const int64_t dyn_base = S * gridDim.x;
+        const int64_t dyn_n = total - dyn_base;
+        int64_t stat_next = S * blockIdx.x;
+        const int64_t stat_end = stat_next + S;
+        // lane 0: the next dynamic ticket, fetched one piece ahead (-1: none yet)
+        int64_t ticket = -1;
+        bool tickets_done = false;
+        auto take_ticket = [&]() {
+            ticket = dyn_n > 0 ? int64_t(atomicAdd(p.dyn_ticket, 1)) : dyn_n;
+        };
+        // lane 0: the next piece to issue, or -1 when there is none
+        auto next_piece = [&]() -> int64_t {
+            if (stat_next < stat_end) {
+                const int64_t pc = stat_next++;
+                if (stat_next == stat_end && !tickets_done && ticket < 0) take_ticket();
+                return pc;
+            }
+            if (tickets_done) return -1;
+            if (ticket < 0) take_ticket();
+            if (ticket >= dyn_n) {
+                tickets_done = true;
+                return -1;
+            }
+            const int64_t pc = dyn_base + ticket;
+            take_ticket();
+            return pc;
+        };
+        int64_t cur = lane == 0 ? next_piece() : -1;
+        int issued = 0, merged = 0;
+        bool end_sent = false, stop = false;
         int last_round[kStages];    // round of the last copy issued into each stage, -1 = none
 #pragma unroll
         for (int s = 0; s < kStages; ++s) last_round[s] = -1;
-        bool stop = false;
-        while (merged < hi) {
-            if (next < hi && next - merged < kStages) {
-                const int64_t k = next - lo;
-                const int slot = static_cast<int>(k % kStages);
-                const int round = static_cast<int>(k / kStages);
-                if (lane == 0) {
-                    const ItemDesc d = decode_item<T>(p, row_start, next);
+        // lane 0: issue the next item (piece `cur`, or the end marker) into its stage
+        auto issue_next = [&]() {
+            const int slot = issued % kStages;
+            const int round = issued / kStages;
+            if (lane == 0) {
+                StageMeta m;
+                if (cur >= 0) {
+                    const ItemDesc d = decode_item<T>(p, row_start, cur);
                     const int64_t bytes_all = int64_t(d.e1 - d.e0) * Logit<T>::kSize;
                     const int n = static_cast<int>(bytes_all & ~int64_t(15));
                     const int tail_n = static_cast<int>((bytes_all - n) / Logit<T>::kSize);
                     const unsigned char* src = d.row + int64_t(d.e0) * Logit<T>::kSize;
+                    m.tail = tail_n ? src + n : nullptr;
+                    m.partial_idx = d.partial_idx;
+                    m.elem0 = d.e0;
+                    m.n_bytes = n;
+                    m.tail_n = tail_n;
+                    m.pad = 0;
+                    meta[slot] = m;
                     if (d.partial_idx == p.lost_copy_partial) {
                         // injected fault: the stage is neither armed nor copied, so
                         // the consumers' bounded wait on it runs out
                     } else {
-                        StageMeta m;
-                        m.tail = tail_n ? src + n : nullptr;
-                        m.partial_idx = d.partial_idx;
-                        m.elem0 = d.e0;
-                        m.n_bytes = n;
-                        m.tail_n = tail_n;
-                        m.pad = 0;
-                        meta[slot] = m;
 #pragma unroll
                         for (int s = 0; s < kStages; ++s)
                             if (s == slot) last_round[s] = round;
                         if (n > 0) {
                             mbar_arrive_expect_tx(full + slot, static_cast<uint32_t>(n));
-                            bulk_copy_g2s(stage_buf + size_t(slot) * kStageBytes, src, static_cast<uint32_t>(n),
-                                          full + slot);
+                            bulk_copy_g2s_hint(stage_buf + size_t(slot) * kStageBytes, src, static_cast<uint32_t>(n),
+                                               full + slot, stream_policy);
                         } else {
                             mbar_arrive(full + slot);
                         }
                     }
+                    cur = next_piece();
+                } else {
+                    m.tail = nullptr;
+                    m.partial_idx = -1;
+                    m.elem0 = 0;
+                    m.n_bytes = -1;
+                    m.tail_n = 0;
+                    m.pad = 0;
+                    meta[slot] = m;
+                    mbar_arrive(full + slot);
                 }
-                ++next;
+            }
+        };
+        for (;;) {
+            if (!end_sent && issued - merged < kStages) {
+                const bool has_piece = __shfl_sync(0xffffffffu, cur >= 0, 0);
+                issue_next();
+                if (!has_piece) end_sent = true;
+                ++issued;
                 continue;
             }
-            const int64_t k = merged - lo;
-            const int slot = static_cast<int>(k % kStages);
-            const int round = static_cast<int>(k / kStages);
+            const int n_real = issued - (end_sent ? 1 : 0);
+            if (merged == n_real) break;
+            const int slot = merged % kStages;
+            const int round = merged / kStages;
             bool ok = true;
             if (lane == 0) ok = mbar_wait_or_abort(empty + slot, static_cast<uint32_t>(round & 1), p.timeout_ns,
                                                    abort_flag);
@@ -536,20 +587,37 @@ row_stats_tma_kernel(const StatsParams p) {
                 stop = true;
                 break;
             }
+            // the piece's partial index, read before the refill rewrites meta[slot]
+            const int64_t pidx = meta[slot].partial_idx;
+            __syncwarp();
+            ++merged;
+            if (!end_sent && issued - merged < kStages) {
+                const bool has_piece = __shfl_sync(0xffffffffu, cur >= 0, 0);
+                issue_next();
+                if (!has_piece) end_sent = true;
+                ++issued;
+            }
             float2 v[kPartsPerLane];
-            const float2* ps = part + slot * kConsumers;
+            const float2* ps = part + ((round & 1) * kStages + slot) * kConsumers;
 #pragma unroll
             for (int i = 0; i < kPartsPerLane; ++i) v[i] = ps[lane + 32 * i];
             const float2 r = warp_merge_parts<kGreedy, kPartsPerLane>(v);
-            if (lane == 0) p.partials[meta[slot].partial_idx] = r;
-            ++merged;
+            if (lane == 0) p.partials[pidx] = r;
         }
-        if (stop) {
-            // the pieces left unmerged get NaN partials: the scan kernel reports
-            // their requests with out_accept_len = -2
+        if (stop && lane == 0) {
+            // every piece this CTA took and did not finish gets a NaN partial
+            // (the scan kernel reports its request with out_accept_len = -2):
+            // the pieces in the ring, the rest of the static range, the piece
+            // about to be issued and the ticket fetched ahead
             const float nan = __int_as_float(0x7fc00000);
-            for (int64_t it = merged + lane; it < hi; it += 32)
-                p.partials[decode_item<T>(p, row_start, it).partial_idx] = make_float2(nan, nan);
+            const float2 bad = make_float2(nan, nan);
+            const int n_real = issued - (end_sent ? 1 : 0);
+            for (int i = merged; i < n_real; ++i) p.partials[meta[i % kStages].partial_idx] = bad;
+            for (int64_t it = stat_next; it < stat_end; ++it)
+                p.partials[decode_item<T>(p, row_start, it).partial_idx] = bad;
+            if (cur >= 0) p.partials[decode_item<T>(p, row_start, cur).partial_idx] = bad;
+            if (!tickets_done && ticket >= 0 && ticket < dyn_n)
+                p.partials[decode_item<T>(p, row_start, dyn_base + ticket).partial_idx] = bad;
         }
         // Wait until the consumers are done, then make sure no copy issued by
         // this CTA is still in flight before exiting (after a timeout).
@@ -564,22 +632,24 @@ row_stats_tma_kernel(const StatsParams p) {
     }
 
     // ------------------------------- consumer warps -------------------------------
-    // Each piece: wait for its stage, fold it (plus the row's ragged tail on
-    // the row's last piece), leave this thread's partial in part[stage][tid]
-    // and release the stage.  A failed wait is made warp-uniform; the warp
-    // then leaves the loop (the producer writes the NaN partials).
+    // Item i: wait for its stage, stop at the end marker, else fold the piece
+    // (plus the row's ragged tail on the row's last piece), leave this
+    // thread's partial in part[round & 1][stage][tid] and release the stage.
+    // A failed wait is made warp-uniform; the warp then leaves the loop (the
+    // producer writes the NaN partials).
     const int lane = tid & 31;
-    for (int64_t piece = lo; piece < hi; ++piece) {
-        const int64_t k = piece - lo;
-        const int slot = static_cast<int>(k % kStages);
-        const uint32_t parity = static_cast<uint32_t>((k / kStages) & 1);
-        bool ok = !*abort_flag && mbar_wait_or_abort(full + slot, parity, p.timeout_ns, abort_flag);
+    for (int i = 0;; ++i) {
+        const int slot = i % kStages;
+        const int round = i / kStages;
+        bool ok = !*abort_flag && mbar_wait_or_abort(full + slot, static_cast<uint32_t>(round & 1), p.timeout_ns,
+                                                     abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) {
             if (lane == 0) *abort_flag = 1;
             break;
         }
         const StageMeta m = meta[slot];
+        if (m.n_bytes < 0) break;  // end marker: no more pieces
         const unsigned char* buf = stage_buf + size_t(slot) * kStageBytes;
         const int nvec = m.n_bytes >> 4;
         Acc<kGreedy> acc;
@@ -613,13 +683,11 @@ row_stats_tma_kernel(const StatsParams p) {
             if constexpr (kGreedy) acc.take(z, idx);
             else acc.fold1(z * p.scale);
         }
-        part[slot * kConsumers + tid] = acc.as_float2();
+        part[((round & 1) * kStages + slot) * kConsumers + tid] = acc.as_float2();
         __syncwarp();
         if (lane == 0) mbar_arrive(empty + slot);  // release: the partials above are visible to the producer
     }
     named_barrier_sync(2, kThreads);
-    // this CTA is done: the dependent scan kernel may start its prologue here
-    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
 }
 
 // ============================================================================
@@ -633,7 +701,7 @@ row_stats_ldg_kernel(const StatsParams p) {
     extern __shared__ __align__(16) int ldg_row_start[];
     __shared__ int scan_scratch[32];
     __shared__ float red[2][2 * kWarps];
-    zero_ctrl(p);
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;");  // see the bulk-copy variant
     build_row_prefix<kThreads>(p, ldg_row_start, scan_scratch);
     int64_t lo, hi;
     piece_range((int64_t)ldg_row_start[p.nB] * p.P, &lo, &hi);
@@ -691,8 +759,6 @@ row_stats_ldg_kernel(const StatsParams p) {
         }
         reduce_and_store<kGreedy, kWarps>(acc, red[parity_item], 1, kThreads, p.partials + d.partial_idx);
     }
-    __syncthreads();
-    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
 }
 
 }  // namespace sv

@@ -1,13 +1,15 @@
-// sv_verify_draw.cuh -- K2b, the final draw (residual / bonus / one-hot).
+// sv_verify_draw.cuh -- K2b, the final draw (residual / bonus / one-hot),
+// and K2c, the selection of residual draws.
 //
 // The scan kernel queued one draw per sampling request: a residual draw
 // (rejection with draft logits) as P tasks, one per piece of the row pair,
-// and a bonus or one-hot draw as one task.  This kernel is a persistent grid
-// of resident CTAs; CTA x takes tasks x, x + G, x + 2G, ... (residual tasks
+// and a bonus or one-hot draw as one task.  K2b is a persistent grid of
+// resident CTAs; CTA x takes tasks x, x + G, x + 2G, ... (residual tasks
 // first, ordered slot-major, so one draw's pieces run on P different CTAs at
 // once).  Each task stages its piece(s) in shared memory with 1-D bulk copies
-// (double-buffered: the next task's copies are in flight while the current
-// one is computed) and computes the draw weights
+// (double-buffered: the next task's copies, and the queue entry of the one
+// after, are in flight while the current task is computed) and computes the
+// draw weights
 //     residual: w_v = max(0, p_j(v) - q_j(v))     ("AI 开始抄自己的作业——而且抄得理直气壮",
 //               section "⚡ 投机解码：让草稿先跑，考官殿后": the redraw comes from the
 //               target with the draft's share taken out);
@@ -21,11 +23,10 @@
 // The token is the smallest v whose running weight sum exceeds u*W (u* =
 // uniforms[b][k_max], W the total); it is found piece -> segment -> vector ->
 // element:
-//   * residual: each task stores its piece's 32 segment sums and counts the
-//     piece as done (atomic add after a fence); the CTA that finishes the
-//     last piece picks the piece and segment from the stored sums, re-reads
-//     that one segment of both rows (one vector per lane) and picks the
-//     vector and element.  Nothing waits on another CTA.
+//   * residual: each K2b task stores its piece's 32 segment sums; K2c (one
+//     warp per residual draw, after K2b) picks the piece and the segment from
+//     the stored sums, re-reads that one segment of both rows (one vector per
+//     lane) and picks the vector and element.  Nothing waits on another CTA.
 //   * bonus: the piece was chosen by the scan kernel from the row-statistics
 //     partials; the task picks segment, vector and element in shared memory.
 //   * one-hot: the task computes the exact weight of the piece holding the
@@ -36,7 +37,7 @@
 // block with positive weight there, so a zero-weight token is never drawn.
 // A zero residual mass (p == q numerically) draws from p_j instead.
 //
-// Waits: only on this CTA's own bulk copies, bounded by timeout_ns; after a
+// Waits: only on a CTA's own bulk copies, bounded by timeout_ns; after a
 // timeout the CTA reports its remaining draws with out_accept_len = -2.
 #pragma once
 
@@ -50,13 +51,14 @@
 namespace sv {
 
 struct DrawParams {
+    int32_t B;
     const unsigned char* target;
     const unsigned char* draft;
     const float2* partials;      // [B][2k+1][P] row-statistics partials
     const int32_t* ctrl;         // [0] residual draws, [1] single-piece draws
     const DrawReq* res_req;
     const DrawReq* one_req;
-    int32_t* res_cnt;            // [B] pieces finished per residual draw
+    int32_t* res_lost;           // [B] per residual draw: set when one of its pieces was lost to a timeout
     float* seg;                  // [B][P][32] segment sums of residual draws (by queue slot)
     int32_t* out_len;
     int32_t* out_tokens;
@@ -152,26 +154,95 @@ __device__ __forceinline__ float piece_vec_weights(const WeightRow& r, const uns
     return vec_weights<T>(r, z, y, idx0, count, w);
 }
 
+// Sum of the draw weights of one whole staged vector (PV elements from row
+// index idx0), for a draw of mode kMode; every element weight is computed
+// exactly as vec_weights computes it (the selection recomputes them there).
+// A one-hot vector holding the drafted id goes through vec_weights, so the
+// drafted id's weight is left out rather than subtracted.
+template <typename T, int kMode>
+__device__ __forceinline__ float vec_sum_staged(const WeightRow& r, const unsigned char* tp, const unsigned char* dp,
+                                                int idx0) {
+    constexpr int PV = Logit<T>::kPerVec;
+    float z[PV], y[PV];
+    Logit<T>::unpack(ld_shared_v4(tp), z);
+    if constexpr (kMode == kResidual) Logit<T>::unpack(ld_shared_v4(dp), y);
+    if constexpr (kMode == kOneHot) {
+        if (static_cast<unsigned>(r.zero_at - idx0) < static_cast<unsigned>(PV)) {
+            float w[PV];
+#pragma unroll
+            for (int i = 0; i < PV; ++i) y[i] = 0.f;
+            return vec_weights<T>(r, z, y, idx0, PV, w);
+        }
+    }
+    const float nlp = -r.lse_p, nlq = -r.lse_q;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < PV; i += 2) {
+        float w0 = ex2_approx(fmaf(z[i], r.scale, nlp));
+        float w1 = ex2_approx(fmaf(z[i + 1], r.scale, nlp));
+        if constexpr (kMode == kResidual) {
+            w0 = fmaxf(0.f, w0 - ex2_approx(fmaf(y[i], r.scale, nlq)));
+            w1 = fmaxf(0.f, w1 - ex2_approx(fmaf(y[i + 1], r.scale, nlq)));
+        }
+        s0 += w0;
+        s1 += w1;
+    }
+    return s0 + s1;
+}
+
 // All threads: the 32 segment sums of one piece into s_seg (ends with
 // __syncthreads).  Thread t handles vectors t + 256 k, so warp w at step k
-// covers segment w + 8 k.
+// covers segment w + 8 k.  Whole staged vectors take the fast path; the
+// ragged end of a row and unstaged (unaligned) rows take the general one.
+template <typename T, int kMode>
+__device__ __forceinline__ void piece_segments_mode(const WeightRow& r, const unsigned char* tbuf,
+                                                    const unsigned char* dbuf, int nstaged_vec, bool vec_ok, int e0,
+                                                    int n, float* s_seg) {
+    constexpr int PV = Logit<T>::kPerVec;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nvec = (n + PV - 1) / PV;
+    float sum[kVecsPerThread];
+    if (nstaged_vec == kPieceVecs) {
+        // a whole staged piece: every vector on the fast path, all in flight
+#pragma unroll
+        for (int k = 0; k < kVecsPerThread; ++k) {
+            const int v = threadIdx.x + k * kDrawThreads;
+            sum[k] = vec_sum_staged<T, kMode>(r, tbuf + 16 * v, kMode == kResidual ? dbuf + 16 * v : nullptr,
+                                              e0 + v * PV);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < kVecsPerThread; ++k) {
+            const int v = threadIdx.x + k * kDrawThreads;
+            sum[k] = 0.f;
+            if (v < nstaged_vec) {
+                sum[k] = vec_sum_staged<T, kMode>(r, tbuf + 16 * v, kMode == kResidual ? dbuf + 16 * v : nullptr,
+                                                  e0 + v * PV);
+            } else if (v < nvec) {
+                float w[PV];
+                sum[k] = piece_vec_weights<T>(r, tbuf, dbuf, nstaged_vec, vec_ok, e0, n, v, w);
+            }
+        }
+    }
+    // four independent warp sums, interleaved
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int k = 0; k < kVecsPerThread; ++k) sum[k] += __shfl_xor_sync(0xffffffffu, sum[k], o);
+    if (lane == 0) {
+#pragma unroll
+        for (int k = 0; k < kVecsPerThread; ++k) s_seg[warp + kDrawWarps * k] = sum[k];
+    }
+    __syncthreads();
+}
+
 template <typename T>
 __device__ __forceinline__ void piece_segments(const WeightRow& r, const unsigned char* tbuf,
                                                const unsigned char* dbuf, int nstaged_vec, bool vec_ok, int e0,
                                                int n, float* s_seg) {
-    constexpr int PV = Logit<T>::kPerVec;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nvec = (n + PV - 1) / PV;
-#pragma unroll
-    for (int k = 0; k < kVecsPerThread; ++k) {
-        const int v = threadIdx.x + k * kDrawThreads;
-        float w[PV];
-        float sum = v < nvec ? piece_vec_weights<T>(r, tbuf, dbuf, nstaged_vec, vec_ok, e0, n, v, w) : 0.f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) s_seg[warp + kDrawWarps * k] = sum;
-    }
-    __syncthreads();
+    if (r.mode == kResidual) piece_segments_mode<T, kResidual>(r, tbuf, dbuf, nstaged_vec, vec_ok, e0, n, s_seg);
+    else if (r.mode == kOneHot) piece_segments_mode<T, kOneHot>(r, tbuf, dbuf, nstaged_vec, vec_ok, e0, n, s_seg);
+    else piece_segments_mode<T, kBonus>(r, tbuf, dbuf, nstaged_vec, vec_ok, e0, n, s_seg);
 }
 
 // One warp: inside a piece (elements [e0, e0 + n) of row j) whose segment
@@ -253,6 +324,11 @@ __device__ __forceinline__ void pick_piece(const float* s_pw, int P, float ustar
     }
 }
 
+// The draw of task t: a queue entry, and the piece it stages first.
+__device__ __forceinline__ DrawReq task_req(const DrawParams& p, int64_t t, int64_t n_res_tasks) {
+    return t < n_res_tasks ? load_req(p.res_req + t / p.P) : load_req(p.one_req + (t - n_res_tasks));
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kDrawThreads, kDrawCtasPerSm)
 verify_draw_kernel(const DrawParams p) {
@@ -261,7 +337,7 @@ verify_draw_kernel(const DrawParams p) {
     __shared__ float s_seg[kSegsPerPiece];
     __shared__ float s_pw[kMaxPieces];
     __shared__ DrawReq s_req[2];
-    __shared__ int s_last, s_pick;
+    __shared__ int s_pick;
     __shared__ float s_target, s_W;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -270,8 +346,14 @@ verify_draw_kernel(const DrawParams p) {
     const int64_t esz = Logit<T>::kSize;
     const bool vec_ok = p.rows_aligned != 0;
 
-    // the scan kernel's queue (this kernel is a programmatic dependent of it)
+    // the selection kernel may be launched now; it waits for this grid
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
+    // the scan kernel's queue (this kernel is a programmatic dependent of it);
+    // thread 0 reads its first task's entry together with the queue lengths,
+    // taking it to be a residual piece (it is, unless few draws are residual)
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    DrawReq first;
+    if (tid == 0) first = load_req(p.res_req + min(int(blockIdx.x / P), p.B - 1));
     const int nres = __ldcg(p.ctrl + 0);
     const int none = __ldcg(p.ctrl + 1);
     const int64_t n_res_tasks = int64_t(nres) * P;
@@ -299,21 +381,11 @@ verify_draw_kernel(const DrawParams p) {
     bool pend0 = false, pend1 = false;
     bool failed = false;  // a wait ran out: every later draw of this CTA is reported -2
 
-    // Thread 0 only: read task t's draw into s_req[buf] and issue the copies
+    // Thread 0 only: store task t's draw r in s_req[buf] and issue the copies
     // of its first piece into buffer buf (completing on s_bar[buf]).
-    auto issue = [&](int64_t t, int buf) {
-        DrawReq r;
-        int pc;
-        bool resid;
-        if (t < n_res_tasks) {
-            r = load_req(p.res_req + t / P);
-            pc = static_cast<int>(t % P);
-            resid = true;
-        } else {
-            r = load_req(p.one_req + (t - n_res_tasks));
-            pc = r.mode == kBonus ? r.piece : r.x / p.PE;
-            resid = false;
-        }
+    auto issue = [&](int64_t t, const DrawReq& r, int buf) {
+        const bool resid = t < n_res_tasks;
+        const int pc = resid ? static_cast<int>(t % P) : (r.mode == kBonus ? r.piece : r.x / p.PE);
         s_req[buf] = r;
         if (r.b == p.lost_draw_b && pc == (resid ? 0 : pc)) return;  // injected fault: nothing completes the wait
         unsigned char* dst = draw_dsm + size_t(buf) * kDrawBufBytes;
@@ -324,8 +396,9 @@ verify_draw_kernel(const DrawParams p) {
         }
         mbar_arrive_expect_tx(&s_bar[buf], resid ? 2 * nb : nb);
         const int64_t off = int64_t(pc) * p.PE * esz;
-        bulk_copy_g2s(dst, trow_of(r) + off, nb, &s_bar[buf]);
-        if (resid) bulk_copy_g2s(dst + kPieceBytes, drow_of(r) + off, nb, &s_bar[buf]);
+        const uint64_t pol = l2_evict_first_policy();  // each piece is staged once
+        bulk_copy_g2s_hint(dst, trow_of(r) + off, nb, &s_bar[buf], pol);
+        if (resid) bulk_copy_g2s_hint(dst + kPieceBytes, drow_of(r) + off, nb, &s_bar[buf], pol);
     };
     // All threads: wait for buffer buf's pending completion (bounded);
     // block-uniform result.  On success the parity moves on; on a timeout it
@@ -339,13 +412,25 @@ verify_draw_kernel(const DrawParams p) {
         }
         return ok;
     };
-    auto fail_request = [&](const DrawReq& r) {
+    // A lost draw: the request reports -2; a residual draw is also marked so
+    // that the selection kernel leaves it alone.
+    auto fail_request = [&](const DrawReq& r, int64_t t) {
         int32_t* tok = p.out_tokens + int64_t(r.b) * (K + 1);
         for (int i = tid; i <= K; i += kDrawThreads) tok[i] = -1;
-        if (tid == 0) p.out_len[r.b] = -2;
+        if (tid == 0) {
+            p.out_len[r.b] = -2;
+            if (t < n_res_tasks) p.res_lost[t / P] = 1;
+        }
     };
 
-    if (tid == 0) issue(blockIdx.x, 0);
+    // Thread 0 keeps the queue entry of the task after the next one in
+    // registers, loaded one iteration ahead of its use.
+    DrawReq ahead;
+    if (tid == 0) {
+        if (int64_t(blockIdx.x) >= n_res_tasks) first = task_req(p, blockIdx.x, n_res_tasks);
+        issue(blockIdx.x, first, 0);
+        if (blockIdx.x + gridDim.x < ntask) ahead = task_req(p, blockIdx.x + gridDim.x, n_res_tasks);
+    }
     pend0 = true;
     int it = 0;
     for (int64_t t = blockIdx.x; t < ntask; t += gridDim.x, ++it) {
@@ -353,24 +438,23 @@ verify_draw_kernel(const DrawParams p) {
         const int64_t tn = t + gridDim.x;
         __syncthreads();  // s_req[buf] is written; buffer buf ^ 1 is free again
         const DrawReq r = s_req[buf];
-        if (failed) {
-            fail_request(r);
-            if (tn < ntask && tid == 0) s_req[buf ^ 1] = t + gridDim.x < n_res_tasks
-                                                             ? load_req(p.res_req + tn / P)
-                                                             : load_req(p.one_req + (tn - n_res_tasks));
-            continue;
-        }
         if (tn < ntask) {
-            if (tid == 0) issue(tn, buf ^ 1);
-            if (buf) pend0 = true; else pend1 = true;
+            if (tid == 0) {
+                if (failed) s_req[buf ^ 1] = ahead;   // no more copies: only the entry is passed on
+                else issue(tn, ahead, buf ^ 1);
+                if (tn + gridDim.x < ntask) ahead = task_req(p, tn + gridDim.x, n_res_tasks);
+            }
+            if (!failed) {
+                if (buf) pend0 = true; else pend1 = true;
+            }
+        }
+        if (failed) {
+            fail_request(r, t);
+            continue;
         }
         if (!wait_buf(buf)) {
             failed = true;
-            fail_request(r);
-            if (tn < ntask && tid == 0) {
-                // the next task's draw is already in s_req[buf ^ 1]; its copy is
-                // pending and drained at the end
-            }
+            fail_request(r, t);
             continue;
         }
         unsigned char* tbuf = draw_dsm + size_t(buf) * kDrawBufBytes;
@@ -387,56 +471,14 @@ verify_draw_kernel(const DrawParams p) {
         int pc_loaded = -1;   // piece of target row j staged in tbuf with s_seg holding its p-based segment sums
 
         if (t < n_res_tasks) {
-            // ---------------------------- residual piece ----------------------------
+            // residual piece: its segment sums go to the selection kernel
             const int slot = static_cast<int>(t / P);
             const int pc = static_cast<int>(t % P);
             piece_segments<T>(wr, tbuf, dbuf, staged_bytes(pc) / 16, vec_ok, pc * p.PE, piece_n(pc), s_seg);
-            float* seg_out = p.seg + (int64_t(slot) * P + pc) * kSegsPerPiece;
-            if (warp == 0) {
-                seg_out[lane] = s_seg[lane];
-                __threadfence();  // the sums are visible before the piece is counted
-            }
-            __syncthreads();
-            if (tid == 0) {
-                s_last = atomicAdd(p.res_cnt + slot, 1) == P - 1;
-                __threadfence();
-            }
-            __syncthreads();
-            if (!s_last) continue;
-            // The last piece of this draw: piece totals from every task's
-            // segment sums, then piece, segment (sums re-read into s_seg) and
-            // element (one vector per lane re-read from the rows).
-            const float* seg_all = p.seg + int64_t(slot) * P * kSegsPerPiece;
-            for (int c = warp; c < P; c += kDrawWarps) {
-                float v = __ldcg(seg_all + int64_t(c) * kSegsPerPiece + lane);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) s_pw[c] = v;
-            }
-            __syncthreads();
-            if (warp == 0) pick_piece(s_pw, P, r.ustar, &s_pick, &s_target, &s_W);
-            __syncthreads();
-            if (s_W > 0.f) {
-                const int pstar = s_pick;
-                if (warp == 0) {
-                    s_seg[lane] = __ldcg(seg_all + int64_t(pstar) * kSegsPerPiece + lane);
-                    __syncwarp();
-                    const int tok = select_in_piece<T>(wr, s_seg, nullptr, nullptr, 0, vec_ok, pstar * p.PE,
-                                                       piece_n(pstar), s_target);
-                    if (lane == 0) s_pick = tok;
-                }
-                __syncthreads();
-                if (s_pick >= 0) {
-                    if (tid == 0) *out_tok = s_pick;
-                } else {
-                    fail_request(r);
-                }
-                continue;
-            }
-            // zero residual mass (p == q numerically): the draw uses p_j
-            wr.mode = kBonus;
-            wr.drow = nullptr;
-        } else if (r.mode == kBonus) {
+            if (warp == 0) p.seg[(int64_t(slot) * P + pc) * kSegsPerPiece + lane] = s_seg[lane];
+            continue;
+        }
+        if (r.mode == kBonus) {
             // ------------------ bonus: the scan kernel chose the piece ------------------
             piece_segments<T>(wr, tbuf, nullptr, staged_bytes(r.piece) / 16, vec_ok, r.piece * p.PE,
                               piece_n(r.piece), s_seg);
@@ -548,7 +590,7 @@ verify_draw_kernel(const DrawParams p) {
         if (tok >= 0) {
             if (tid == 0) *out_tok = tok;
         } else {
-            fail_request(r);
+            fail_request(r, t);
         }
     }
     // A copy issued into a buffer that was never (successfully) waited for
@@ -557,6 +599,139 @@ verify_draw_kernel(const DrawParams p) {
     if (tid == 0) {
         if (pend0) (void)mbar_wait_bounded(&s_bar[0], ph0, p.timeout_ns);
         if (pend1) (void)mbar_wait_bounded(&s_bar[1], ph1, p.timeout_ns);
+    }
+}
+
+// ============================================================================
+// K2c: selection of the residual draws, one warp per queued residual draw.
+
+constexpr int kSelectThreads = 256;
+constexpr int kSelectWarps = kSelectThreads / 32;
+
+struct SelectParams {
+    int32_t B;
+    const unsigned char* target;
+    const unsigned char* draft;
+    const float2* partials;
+    const int32_t* ctrl;
+    const DrawReq* res_req;
+    const float* seg;            // [B][P][32] segment sums written by K2b
+    const int32_t* res_lost;     // [B] residual draws K2b lost to a timeout (already reported -2)
+    int32_t* out_len;
+    int32_t* out_tokens;
+    int32_t k_max;
+    int32_t V;
+    int64_t row_stride;
+    int32_t P;
+    int32_t PE;
+    float scale;
+    int32_t rows_aligned;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kSelectThreads)
+verify_select_kernel(const SelectParams p) {
+    constexpr int PV = Logit<T>::kPerVec;
+    __shared__ float s_segs[kSelectWarps][kSegsPerPiece];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // slot < B: every load below stays inside the workspace, so the queue
+    // length, the loss mark, the entry and the segment sums are read at once
+    const int slot = blockIdx.x * kSelectWarps + warp;
+    if (slot >= p.B) return;
+    const int K = p.k_max;
+    const int P = p.P;
+    const int64_t esz = Logit<T>::kSize;
+    const bool vec_ok = p.rows_aligned != 0;
+    const int nres = __ldcg(p.ctrl + 0);
+    const int lost = __ldcg(p.res_lost + slot);
+    const DrawReq r = load_req(p.res_req + slot);
+    WeightRow wr;
+    wr.trow = p.target + (int64_t(r.b) * (K + 1) + r.j) * p.row_stride * esz;
+    wr.drow = p.draft + (int64_t(r.b) * K + r.j) * p.row_stride * esz;
+    wr.scale = p.scale;
+    wr.lse_p = r.lse_p;
+    wr.lse_q = r.lse_q;
+    wr.mode = kResidual;
+    wr.zero_at = -1;
+    const float* seg = p.seg + int64_t(slot) * P * kSegsPerPiece;
+    // piece totals: lane l sums the 32 segment sums of its pieces [l*cps, l*cps + cps)
+    const int cps = (P + 31) / 32;
+    float w[kMaxPiecesPerLane];
+#pragma unroll
+    for (int k = 0; k < kMaxPiecesPerLane; ++k) {
+        const int c = lane * cps + k;
+        float t = 0.f;
+        if (k < cps && c < P) {
+            const float4* s4 = reinterpret_cast<const float4*>(seg + int64_t(c) * kSegsPerPiece);
+#pragma unroll
+            for (int q = 0; q < kSegsPerPiece / 4; ++q) {
+                const float4 v = s4[q];
+                t += (v.x + v.y) + (v.z + v.w);
+            }
+        }
+        w[k] = t;
+    }
+    if (slot >= nres || lost != 0) return;
+    float tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMaxPiecesPerLane; ++k) tot += w[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    float local = INFINITY;
+    int pstar = -1;
+    const float* segp = nullptr;
+    if (tot > 0.f) {
+        pstar = warp_pick<kMaxPiecesPerLane>(w, P, r.ustar * tot, &local);
+        segp = seg + int64_t(pstar) * kSegsPerPiece;
+    } else {
+        // zero residual mass (p == q numerically): draw from p_j -- the piece
+        // from the partials, its segment sums computed here by the warp
+        wr.mode = kBonus;
+        wr.drow = nullptr;
+        const float2* part_j = p.partials + (int64_t(r.b) * (2 * K + 1) + r.j) * P;
+        float pw[kMaxPiecesPerLane];
+        float ptot = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxPiecesPerLane; ++k) {
+            const int c = lane * cps + k;
+            pw[k] = 0.f;
+            if (k < cps && c < P) {
+                const float2 pp = part_j[c];
+                pw[k] = pp.y * exp2f(pp.x - wr.lse_p);
+            }
+            ptot += pw[k];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ptot += __shfl_xor_sync(0xffffffffu, ptot, o);
+        if (ptot > 0.f) pstar = warp_pick<kMaxPiecesPerLane>(pw, P, r.ustar * ptot, &local);
+        if (pstar >= 0) {
+            const int e0 = pstar * p.PE, n = min(p.V - e0, p.PE);
+            const int nvec = (n + PV - 1) / PV;
+            for (int sg = 0; sg < kSegsPerPiece; ++sg) {
+                const int v = sg * kSegVecs + lane;
+                float wv[PV];
+                float sum = v < nvec ? piece_vec_weights<T>(wr, nullptr, nullptr, 0, vec_ok, e0, n, v, wv) : 0.f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                if (lane == 0) s_segs[warp][sg] = sum;
+            }
+            __syncwarp();
+            segp = s_segs[warp];
+        }
+    }
+    int tok = -1;
+    if (pstar >= 0)
+        tok = select_in_piece<T>(wr, segp, nullptr, nullptr, 0, vec_ok, pstar * p.PE, min(p.V - pstar * p.PE, p.PE),
+                                 local);
+    if (tok >= 0) {
+        if (lane == 0) p.out_tokens[int64_t(r.b) * (K + 1) + r.j] = tok;
+    } else {
+        // no positive weight anywhere the draw could land (not reached with
+        // finite logits): the request is reported as lost
+        int32_t* out = p.out_tokens + int64_t(r.b) * (K + 1);
+        for (int i = lane; i <= K; i += 32) out[i] = -1;
+        if (lane == 0) p.out_len[r.b] = -2;
     }
 }
 

@@ -67,7 +67,7 @@ struct ScanParams {
     int32_t* ctrl;               // [0] residual draws queued, [1] single-piece draws queued
     DrawReq* res_req;            // [B] residual draws
     DrawReq* one_req;            // [B] bonus / one-hot draws
-    int32_t* res_cnt;            // [B] pieces of each residual draw finished (zeroed here)
+    int32_t* res_lost;           // [B] residual draws lost by the draw kernel (cleared here)
     int32_t k_max;
     int32_t V;
     int64_t row_stride;
@@ -81,11 +81,20 @@ struct ScanParams {
 constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
 constexpr int kMaxDraftsPerThread = (SV_MAX_K + kScanThreads - 1) / kScanThreads;
-constexpr int kMergeRowsPerIter = 4;  // rows per warp with their partial loads in flight together
+constexpr int kMergeRowsPerIter = 8;  // rows per warp with their partial loads in flight together
 
-// Dynamic shared memory: lse_t[k+1] | lse_d[k] | p[k] | q[k]
-__host__ __device__ inline size_t scan_smem_bytes(int k_max) {
+// Dynamic shared memory: lse_t[k+1] | lse_d[k] | p[k] | q[k] | the target
+// rows' partials [k+1][P] (kept for the bonus draw's piece choice when they
+// fit in kScanPartBytes; otherwise that choice reads them again).
+constexpr size_t kScanPartBytes = 24 * 1024;
+__host__ __device__ inline size_t scan_scalar_bytes(int k_max) {
     return (4 * (size_t(k_max + 1) + 3 * size_t(k_max)) + 127) & ~size_t(127);
+}
+__host__ __device__ inline bool scan_keeps_partials(int k_max, int P) {
+    return size_t(k_max + 1) * size_t(P) * 8 <= kScanPartBytes;
+}
+__host__ __device__ inline size_t scan_smem_bytes(int k_max, int P) {
+    return scan_scalar_bytes(k_max) + (scan_keeps_partials(k_max, P) ? size_t(k_max + 1) * size_t(P) * 8 : 0);
 }
 
 // Acceptance probability min(1, p/q); NaN stays NaN (and then rejects).
@@ -176,6 +185,8 @@ verify_scan_kernel(const ScanParams p) {
     float* s_p = s_lse_d + K;   // gathered z(x_i), then p_i
     float* s_q = s_p + K;       // gathered y(x_i), then q_i
     int* s_arg_t = reinterpret_cast<int*>(s_lse_t);  // greedy: argmax per target row
+    const bool keep_parts = !p.greedy && !p.stats_only && scan_keeps_partials(K, P);
+    float2* s_part_t = reinterpret_cast<float2*>(scan_dsm + scan_scalar_bytes(K));  // [L+1][P] when kept
     const int32_t* x = p.tokens + int64_t(b) * K;
     int32_t* out_tok = p.out_tokens ? p.out_tokens + int64_t(b) * (K + 1) : nullptr;
     const bool has_draft = p.draft != nullptr && !p.greedy;
@@ -240,7 +251,6 @@ verify_scan_kernel(const ScanParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (!ok) {
         write_failed(-1);
-        if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
         return;
     }
     if (tid == 0) { s_fail = 0; s_first = L; }
@@ -262,6 +272,17 @@ verify_scan_kernel(const ScanParams p) {
                     const int c = lane + 32 * i;
                     v[rr][i] = (row < nrows && i < per_lane && c < P) ? part_b[int64_t(slot) * P + c]
                                                                       : make_float2(-INFINITY, p.greedy ? __int_as_float(0x7fffffff) : 0.f);
+                }
+            }
+            if (keep_parts) {
+#pragma unroll
+                for (int rr = 0; rr < kMergeRowsPerIter; ++rr) {
+                    const int row = r0 + rr;
+#pragma unroll
+                    for (int i = 0; i < kMaxPiecesPerLane; ++i) {
+                        const int c = lane + 32 * i;
+                        if (row < n_t && c < P) s_part_t[row * P + c] = v[rr][i];
+                    }
                 }
             }
 #pragma unroll
@@ -309,7 +330,6 @@ verify_scan_kernel(const ScanParams p) {
     __syncthreads();
     if (s_fail) {
         write_failed(-2);
-        if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
         return;
     }
 
@@ -362,6 +382,9 @@ verify_scan_kernel(const ScanParams p) {
     }
 
     // 4. outputs of the scan -----------------------------------------------------------
+    // The draw kernel may be launched now (its CTAs then wait for this grid);
+    // launching it earlier would let its waiting CTAs slow this grid down.
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
     const int j = s_first;
     for (int i = tid; i <= K; i += kScanThreads) {
         if (i < j) out_tok[i] = __ldg(x + i);
@@ -387,7 +410,7 @@ verify_scan_kernel(const ScanParams p) {
         if (r.mode == kBonus) {
             // piece weights of p_L from the partials: s * 2^(m - lse); lane l
             // holds pieces [l*cps, l*cps + cps)
-            const float2* part_j = p.partials + (int64_t(b) * nslots + j) * P;
+            const float2* part_j = keep_parts ? s_part_t + j * P : p.partials + (int64_t(b) * nslots + j) * P;
             const int cps = (P + 31) / 32;
             float w[kMaxPiecesPerLane];
 #pragma unroll
@@ -412,7 +435,7 @@ verify_scan_kernel(const ScanParams p) {
         if (lane == 0) {
             if (r.mode == kResidual) {
                 const int slot = atomicAdd(p.ctrl + 0, 1);
-                p.res_cnt[slot] = 0;
+                p.res_lost[slot] = 0;
                 p.res_req[slot] = r;
             } else {
                 const int slot = atomicAdd(p.ctrl + 1, 1);
@@ -420,8 +443,6 @@ verify_scan_kernel(const ScanParams p) {
             }
         }
     }
-    __syncthreads();
-    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
 }
 
 }  // namespace sv

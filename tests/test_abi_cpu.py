@@ -50,12 +50,14 @@ def a256(n):
                                       (4, 4, 1000, sv.F32), (3, 0, 5, sv.BF16), (0, 3, 100, sv.F32)])
 def test_workspace_bytes(B, k, V, dt):
     """Rows are cut into 16 KiB pieces (P per row); the workspace holds one
-    8-byte partial per (request, row slot, piece), a 256-byte control block,
-    two queues of 48-byte draw records, one counter per request and 32
-    segment sums per (request, piece)."""
+    8-byte partial per (request, row slot, piece), the control words (two
+    queue lengths and one piece counter per row-statistics launch of up to
+    4096 requests), two queues of 48-byte draw records, one
+    loss mark per request and 32 segment sums per (request, piece)."""
     es = 2 if dt == sv.BF16 else 4
     P = -(-V * es // PIECE_BYTES)
-    want = (a256(8 * B * (2 * k + 1) * P) + 256 + 2 * a256(48 * B) + a256(4 * B) + a256(4 * 32 * B * P))
+    ctrl = 4 * (2 + -(-B // 4096))
+    want = (a256(8 * B * (2 * k + 1) * P) + a256(ctrl) + 2 * a256(48 * B) + a256(4 * B) + a256(4 * 32 * B * P))
     assert sv.workspace_bytes(B, k, V, dt) == want
 
 
