@@ -251,9 +251,9 @@ __device__ __forceinline__ void piece_segments(const WeightRow& r, const unsigne
 // over lanes) and element.  Returns the row index (same in every lane), or -1
 // when the piece has no positive weight.
 template <typename T>
-__device__ __noinline__ int select_in_piece(const WeightRow r, const float* seg, const unsigned char* tbuf,
-                                            const unsigned char* dbuf, int nstaged_vec, bool vec_ok, int e0, int n,
-                                            float target) {
+__device__ __forceinline__ int select_in_piece_body(const WeightRow& r, const float* seg, const unsigned char* tbuf,
+                                                    const unsigned char* dbuf, int nstaged_vec, bool vec_ok, int e0,
+                                                    int n, float target) {
     constexpr int PV = Logit<T>::kPerVec;
     const int lane = threadIdx.x & 31;
     float one[1] = {seg[lane]};
@@ -287,6 +287,16 @@ __device__ __noinline__ int select_in_piece(const WeightRow r, const float* seg,
         found = e0 + v * PV + (found >= 0 ? found : last);
     }
     return __shfl_sync(0xffffffffu, found, lsel);
+}
+
+// select_in_piece_body as one out-of-line copy (the draw kernel calls it from
+// several places); the selection kernel inlines the body instead, keeping
+// its short code contiguous.
+template <typename T>
+__device__ __noinline__ int select_in_piece(const WeightRow r, const float* seg, const unsigned char* tbuf,
+                                            const unsigned char* dbuf, int nstaged_vec, bool vec_ok, int e0, int n,
+                                            float target) {
+    return select_in_piece_body<T>(r, seg, tbuf, dbuf, nstaged_vec, vec_ok, e0, n, target);
 }
 
 // A queued draw, read through L2 (another kernel wrote it).
@@ -722,8 +732,8 @@ verify_select_kernel(const SelectParams p) {
     }
     int tok = -1;
     if (pstar >= 0)
-        tok = select_in_piece<T>(wr, segp, nullptr, nullptr, 0, vec_ok, pstar * p.PE, min(p.V - pstar * p.PE, p.PE),
-                                 local);
+        tok = select_in_piece_body<T>(wr, segp, nullptr, nullptr, 0, vec_ok, pstar * p.PE,
+                                      min(p.V - pstar * p.PE, p.PE), local);
     if (tok >= 0) {
         if (lane == 0) p.out_tokens[int64_t(r.b) * (K + 1) + r.j] = tok;
     } else {

@@ -81,7 +81,6 @@ struct ScanParams {
 constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
 constexpr int kMaxDraftsPerThread = (SV_MAX_K + kScanThreads - 1) / kScanThreads;
-constexpr int kMergeRowsPerIter = 8;  // rows per warp with their partial loads in flight together
 
 // Dynamic shared memory: lse_t[k+1] | lse_d[k] | p[k] | q[k] | the target
 // rows' partials [k+1][P] (kept for the bonus draw's piece choice when they
@@ -245,9 +244,10 @@ verify_scan_kernel(const ScanParams p) {
     }
 
     // 2. the row-statistics kernel's partials (this kernel is a programmatic
-    // dependent of it: wait for its completion before reading them).  Warp w
-    // merges rows w, w + 8, ..., kMergeRowsPerIter at a time with all their
-    // loads in flight; lane l holds the partials l, l + 32, ... of a row.
+    // dependent of it: wait for its completion before reading them).  Four
+    // lanes merge one row, 64 rows at a time: lane q of a row's group folds
+    // the row's partials q, q + 4, ... (maximum first, then the rescaled
+    // sums), and two shuffles combine the four.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (!ok) {
         write_failed(-1);
@@ -258,70 +258,58 @@ verify_scan_kernel(const ScanParams p) {
     const int n_d = has_draft ? L : 0;
     const int nrows = n_t + n_d;
     {
+        constexpr int kLanesPerRow = 4;
+        constexpr int kRowsPerPass = kScanThreads / kLanesPerRow;
+        constexpr int kMaxPerLane = (kMaxPieces + kLanesPerRow - 1) / kLanesPerRow;
         const float2* part_b = p.partials + int64_t(b) * nslots * P;
-        const int per_lane = (P + 31) / 32;
+        const int q = tid & (kLanesPerRow - 1);
         bool bad = false;
-        for (int r0 = warp * kMergeRowsPerIter; r0 < nrows; r0 += kScanWarps * kMergeRowsPerIter) {
-            float2 v[kMergeRowsPerIter][kMaxPiecesPerLane];
+        for (int r0 = 0; r0 < nrows; r0 += kRowsPerPass) {
+            const int row = r0 + tid / kLanesPerRow;
+            const bool act = row < nrows;
+            const int slot = row < n_t ? row : K + 1 + (row - n_t);
+            const float2* pr = part_b + int64_t(slot) * P;
+            float2 v[kMaxPerLane];
 #pragma unroll
-            for (int rr = 0; rr < kMergeRowsPerIter; ++rr) {
-                const int row = r0 + rr;
-                const int slot = row < n_t ? row : K + 1 + (row - n_t);
-#pragma unroll
-                for (int i = 0; i < kMaxPiecesPerLane; ++i) {
-                    const int c = lane + 32 * i;
-                    v[rr][i] = (row < nrows && i < per_lane && c < P) ? part_b[int64_t(slot) * P + c]
-                                                                      : make_float2(-INFINITY, p.greedy ? __int_as_float(0x7fffffff) : 0.f);
-                }
+            for (int k = 0; k < kMaxPerLane; ++k) {
+                const int c = q + kLanesPerRow * k;
+                v[k] = (act && c < P) ? pr[c] : make_float2(-INFINITY, p.greedy ? __int_as_float(0x7fffffff) : 0.f);
+                if (keep_parts && act && row < n_t && c < P) s_part_t[row * P + c] = v[k];
             }
-            if (keep_parts) {
+            if (p.greedy) {
+                VI r{v[0].x, __float_as_int(v[0].y)};
 #pragma unroll
-                for (int rr = 0; rr < kMergeRowsPerIter; ++rr) {
-                    const int row = r0 + rr;
-#pragma unroll
-                    for (int i = 0; i < kMaxPiecesPerLane; ++i) {
-                        const int c = lane + 32 * i;
-                        if (row < n_t && c < P) s_part_t[row * P + c] = v[rr][i];
+                for (int k = 0; k < kMaxPerLane; ++k) {
+                    if (act && q + kLanesPerRow * k < P) {
+                        const int idx = __float_as_int(v[k].y);
+                        bad |= idx < 0 || idx >= p.V;
                     }
+                    if (k > 0) r = vi_better(r, VI{v[k].x, __float_as_int(v[k].y)});
                 }
-            }
 #pragma unroll
-            for (int rr = 0; rr < kMergeRowsPerIter; ++rr) {
-                const int row = r0 + rr;
-                if (p.greedy) {
-                    VI r{v[rr][0].x, __float_as_int(v[rr][0].y)};
+                for (int o = 1; o < kLanesPerRow; o <<= 1)
+                    r = vi_better(r, VI{__shfl_xor_sync(0xffffffffu, r.v, o), __shfl_xor_sync(0xffffffffu, r.i, o)});
+                if (act && q == 0) s_arg_t[row] = r.i;
+            } else {
+                float m = -INFINITY;
 #pragma unroll
-                    for (int i = 0; i < kMaxPiecesPerLane; ++i) {
-                        const int c = lane + 32 * i;
-                        if (row < nrows && c < P) {
-                            const int idx = __float_as_int(v[rr][i].y);
-                            bad |= idx < 0 || idx >= p.V;
-                        }
-                        if (i > 0) r = vi_better(r, VI{v[rr][i].x, __float_as_int(v[rr][i].y)});
-                    }
-                    r = warp_merge_vi(r);
-                    if (row < nrows && lane == 0) s_arg_t[row] = r.i;
-                } else {
-                    float m = -INFINITY;
+                for (int k = 0; k < kMaxPerLane; ++k) {
+                    bad |= isnan(v[k].x) || isnan(v[k].y);
+                    m = fmaxf(m, v[k].x);
+                }
 #pragma unroll
-                    for (int i = 0; i < kMaxPiecesPerLane; ++i) {
-                        bad |= isnan(v[rr][i].x) || isnan(v[rr][i].y);
-                        m = fmaxf(m, v[rr][i].x);
-                    }
+                for (int o = 1; o < kLanesPerRow; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                float sum = 0.f;
+                if (m != -INFINITY) {
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                    float sum = 0.f;
-                    if (m != -INFINITY) {
+                    for (int k = 0; k < kMaxPerLane; ++k)
+                        if (v[k].x != -INFINITY) sum = fmaf(v[k].y, ex2_approx(v[k].x - m), sum);
+                }
 #pragma unroll
-                        for (int i = 0; i < kMaxPiecesPerLane; ++i)
-                            if (v[rr][i].x != -INFINITY) sum = fmaf(v[rr][i].y, ex2_approx(v[rr][i].x - m), sum);
-                    }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                    if (row < nrows && lane == 0) {
-                        const float lse2 = m + log2f(sum);
-                        if (row < n_t) s_lse_t[row] = lse2; else s_lse_d[row - n_t] = lse2;
-                    }
+                for (int o = 1; o < kLanesPerRow; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                if (act && q == 0) {
+                    const float lse2 = m + log2f(sum);
+                    if (row < n_t) s_lse_t[row] = lse2; else s_lse_d[row - n_t] = lse2;
                 }
             }
         }
