@@ -271,14 +271,23 @@ __device__ __forceinline__ void fold_vectors(Acc<false>& acc, const uint4 (&v)[K
     if (M == -INFINITY) return;
     const float negM = -M;
     float s[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (Logit<T>::kSize == 2) {
+        // Packed pairs: word i's two elements share one FFMA2 and one FADD2
+        // (into {s0, s1} for even i, {s2, s3} for odd i), each lane rounded
+        // as the scalar FFMA and FADD would be.
+        const uint64_t sc2 = f2_pack(scale, scale), nm2 = f2_pack(negM, negM);
+        uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-    for (int i = 0; i < NW; ++i) {
-        if constexpr (Logit<T>::kSize == 2) {
-            s[(2 * i) & 3] += ex2_approx(fmaf(bf16_lo(w[i]), scale, negM));
-            s[(2 * i + 1) & 3] += ex2_approx(fmaf(bf16_hi(w[i]), scale, negM));
-        } else {
-            s[i & 3] += ex2_approx(fmaf(__uint_as_float(w[i]), scale, negM));
+        for (int i = 0; i < NW; ++i) {
+            float xl, xh;
+            f2_unpack(f2_fma(bf16x2_to_f2(w[i]), sc2, nm2), xl, xh);
+            acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(ex2_approx(xl), ex2_approx(xh)));
         }
+        f2_unpack(acc2[0], s[0], s[1]);
+        f2_unpack(acc2[1], s[2], s[3]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) s[i & 3] += ex2_approx(fmaf(__uint_as_float(w[i]), scale, negM));
     }
     acc.ms = MS{M, fmaf(acc.ms.s, ex2_approx(acc.ms.m - M), (s[0] + s[1]) + (s[2] + s[3]))};
 }
