@@ -58,6 +58,7 @@ from speculative_decoding_verification_92_b200.workload import CONFIGS, config_s
 METRIC = "verified draft positions/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 UNIT = "positions/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0                 # B200 HBM3e, vendor figure (context only)
 MAX_REQUESTS_PER_STATS_LAUNCH = 4096     # mirrors the library's launch split
 TRAFFIC_FILE = ROOT / "profiles" / "row_stats_traffic.json"
 
@@ -762,7 +763,11 @@ def run_ours_impl(args):
                 "whole_step_gbs": alg / (ms_per_step / 1e3) / 1e9,
                 "whole_step_frac": alg / (ms_per_step / 1e3) / 1e9 / peak,
                 "reread_bytes_per_step": rr,
-                "whole_step_gbs_with_reread": (alg + rr) / (ms_per_step / 1e3) / 1e9}
+                "whole_step_gbs_with_reread": (alg + rr) / (ms_per_step / 1e3) / 1e9,
+                "whole_step_frac_with_reread": (alg + rr) / (ms_per_step / 1e3) / 1e9 / peak,
+                # context: B200's nominal HBM3e bandwidth (8.0 TB/s), not the denominator
+                "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
+                "whole_step_frac_of_nominal_8000": alg / (ms_per_step / 1e3) / 1e9 / NOMINAL_HBM_GBS}
 
     cfgd = workload_desc(w, args.config)
     cfgd.update({"parallelism": f"replicas{n}" if n > 1 else "single",
