@@ -639,11 +639,11 @@ def reread_bytes(w, g_len, greedy=False) -> int:
     return int((1 + resid.astype(np.int64)).sum()) * w.V * w.esize
 
 
-def launches_per_call(B: int, greedy: bool) -> int:
+def launches_per_call(B: int, greedy: bool, draft_logits: bool) -> int:
     """Kernels one spec_verify call launches: the row-statistics kernel per
-    block of up to 4096 requests, the scan kernel, and (sampling) the draw
-    and selection kernels."""
-    return math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + 1 + (0 if greedy else 2)
+    block of up to 4096 requests, the scan kernel, and for sampling the draw
+    kernel plus (with draft logits: residual draws) the selection kernel."""
+    return math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + 1 + (0 if greedy else 1 + int(draft_logits))
 
 
 def config_record(dw, cfg, steps, warmup, k1_samples, peak):
@@ -800,7 +800,7 @@ def run_ours_impl(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": K, "warmup": W,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic", "config": cfgd,
-            "e2e": e2e, "gpu_launches": K * launches_per_call(w.B, greedy), "roofline": roofline,
+            "e2e": e2e, "gpu_launches": K * launches_per_call(w.B, greedy, w.draft is not None), "roofline": roofline,
             "cpu_baseline": cpu, "clocks": clocks.summary(),
             "hbm_gbs": alg / (ms_per_step / 1e3) / 1e9,
             "accept_rate": accept_rate, "mean_accept_len": float(g_len.mean()),

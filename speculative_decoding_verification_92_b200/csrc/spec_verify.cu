@@ -245,9 +245,9 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
     return cudaSuccess;
 }
 
-// K2a (one CTA per request), then for sampling K2b (persistent, one wave) and
-// K2c (one warp per possible residual draw), each a programmatic dependent of
-// the kernel before it.
+// K2a (one CTA per request), then for sampling K2b (persistent, one wave) and,
+// with draft logits, K2c (one warp per possible residual draw), each a
+// programmatic dependent of the kernel before it.
 template <typename T>
 cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, const SelectParams& cp, int B, bool draw,
                              const DeviceInfo& dev, cudaStream_t st) {
@@ -287,6 +287,8 @@ cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, const S
         cfg.dynamicSmemBytes = kDrawSmemBytes;
         if ((e = cudaLaunchKernelEx(&cfg, k, dp)) != cudaSuccess) return e;
     }
+    // residual draws need draft logits: with one-hot q the queue holds none
+    if (cp.draft == nullptr) return cudaSuccess;
     auto k = verify_select_kernel<T>;
     cfg.gridDim = dim3(static_cast<unsigned>((int64_t(B) + kSelectWarps - 1) / kSelectWarps));
     cfg.blockDim = dim3(kSelectThreads);

@@ -82,12 +82,12 @@ constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
 constexpr int kMaxDraftsPerThread = (SV_MAX_K + kScanThreads - 1) / kScanThreads;
 
-// Dynamic shared memory: lse_t[k+1] | lse_d[k] | p[k] | q[k] | the target
+// Dynamic shared memory: lse_t[k+1] | lse_d[k] | p[k] | q[k] | x[k] | the target
 // rows' partials [k+1][P] (kept for the bonus draw's piece choice when they
 // fit in kScanPartBytes; otherwise that choice reads them again).
 constexpr size_t kScanPartBytes = 24 * 1024;
 __host__ __device__ inline size_t scan_scalar_bytes(int k_max) {
-    return (4 * (size_t(k_max + 1) + 3 * size_t(k_max)) + 127) & ~size_t(127);
+    return (4 * (size_t(k_max + 1) + 4 * size_t(k_max)) + 127) & ~size_t(127);
 }
 __host__ __device__ inline bool scan_keeps_partials(int k_max, int P) {
     return size_t(k_max + 1) * size_t(P) * 8 <= kScanPartBytes;
@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kScanThreads)
 verify_scan_kernel(const ScanParams p) {
     extern __shared__ __align__(128) unsigned char scan_dsm[];
     __shared__ int s_first, s_fail;
+    __shared__ float s_ustar;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.x;
@@ -183,6 +184,7 @@ verify_scan_kernel(const ScanParams p) {
     float* s_lse_d = s_lse_t + (K + 1);
     float* s_p = s_lse_d + K;   // gathered z(x_i), then p_i
     float* s_q = s_p + K;       // gathered y(x_i), then q_i
+    int* s_x = reinterpret_cast<int*>(s_q + K);  // the drafted ids (valid ones only)
     int* s_arg_t = reinterpret_cast<int*>(s_lse_t);  // greedy: argmax per target row
     const bool keep_parts = !p.greedy && !p.stats_only && scan_keeps_partials(K, P);
     float2* s_part_t = reinterpret_cast<float2*>(scan_dsm + scan_scalar_bytes(K));  // [L+1][P] when kept
@@ -226,8 +228,11 @@ verify_scan_kernel(const ScanParams p) {
         if (ok && i < L) {
             xr[k] = __ldg(x + i);
             if (xr[k] < 0 || xr[k] >= p.V) ok = false;
+            s_x[i] = xr[k];
         }
     }
+    // the final draw's uniform, read now so that step 5 waits on no load
+    if (tid == 0 && u && !p.greedy && !p.stats_only) s_ustar = __ldg(u + K);
     ok = __syncthreads_and(ok);
     float ur[kMaxDraftsPerThread];
     if (ok && !p.greedy) {
@@ -375,7 +380,7 @@ verify_scan_kernel(const ScanParams p) {
     if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
     const int j = s_first;
     for (int i = tid; i <= K; i += kScanThreads) {
-        if (i < j) out_tok[i] = __ldg(x + i);
+        if (i < j) out_tok[i] = s_x[i];
         else if (i > j) out_tok[i] = -1;
         else if (p.greedy) out_tok[i] = s_arg_t[j];
     }
@@ -388,11 +393,11 @@ verify_scan_kernel(const ScanParams p) {
         r.b = b;
         r.j = j;
         r.mode = j == L ? kBonus : (has_draft ? kResidual : kOneHot);
-        r.x = j < L ? __ldg(x + j) : -1;
+        r.x = j < L ? s_x[j] : -1;
         r.piece = -1;
         r.lse_p = s_lse_t[j];
         r.lse_q = r.mode == kResidual ? s_lse_d[j] : 0.f;
-        r.ustar = __ldg(u + K);
+        r.ustar = s_ustar;
         r.target = INFINITY;
         r.pad[0] = r.pad[1] = r.pad[2] = 0;
         if (r.mode == kBonus) {
