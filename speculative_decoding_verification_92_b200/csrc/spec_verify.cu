@@ -153,7 +153,7 @@ bool shape_ok(const sv_shape* s, sv_status* why) {
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Control words, zeroed (cudaMemsetAsync) before every call: [0] residual
+// Control words, zeroed (zero_ctrl_kernel) before every call: [0] residual
 // draws queued, [1] one-piece draws queued, [2 + l] the pieces the l-th
 // row-statistics launch (up to 4096 requests each) has handed out.
 int64_t stats_launches(const sv_shape& s) {
@@ -192,6 +192,15 @@ struct NvtxRange {
     ~NvtxRange() { nvtxRangePop(); }
 };
 
+// Zeroes the control words.  It lets the row-statistics kernel launch at
+// once (as its programmatic dependent); that kernel waits for this grid only
+// before its first ticket, so its prologue and first copies overlap this
+// launch.
+__global__ void zero_ctrl_kernel(int32_t* ctrl, int n) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    for (int i = threadIdx.x; i < n; i += blockDim.x) ctrl[i] = 0;
+}
+
 template <typename T, bool kGreedy>
 cudaError_t launch_stats(const StatsParams& base, int B, int variant, const DeviceInfo& dev, cudaStream_t st) {
     for (int b0 = 0; b0 < B; b0 += kMaxRequestsPerLaunch) {
@@ -203,9 +212,11 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
         const int64_t items_upper = int64_t(prm.nB) * rows_max * prm.P;
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.stream = st;
         cfg.attrs = attr;
-        cfg.numAttrs = 0;
+        cfg.numAttrs = 1;
         cudaError_t e;
         if (variant == SV_STATS_TMA) {
             auto k = row_stats_tma_kernel<T, kGreedy, kTmaConsumerWarps, kTmaStages>;
@@ -384,7 +395,8 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     const int lost = a.opts ? a.opts->lost_copy_request : 0;
     sp.lost_copy_partial = lost > 0 ? int64_t(lost - 1) * (2 * s.k_max + 1) * plan.P : -1;
 
-    cudaError_t e = cudaMemsetAsync(ctrl, 0, size_t(ctrl_ints(s)) * sizeof(int32_t), a.stream);
+    zero_ctrl_kernel<<<1, 32, 0, a.stream>>>(ctrl, static_cast<int>(ctrl_ints(s)));
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return SV_ECUDA;
     if (a.opts && a.opts->event_stats_begin)
         if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_begin), a.stream)) != cudaSuccess)

@@ -502,7 +502,14 @@ row_stats_tma_kernel(const StatsParams p) {
         // lane 0: the next dynamic ticket, fetched one piece ahead (-1: none yet)
         int64_t ticket = -1;
         bool tickets_done = false;
+        bool ctrl_ready = false;
         auto take_ticket = [&]() {
+            // the ticket counter is zeroed by the grid this one is a
+            // programmatic dependent of: wait for it before the first ticket
+            if (!ctrl_ready) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                ctrl_ready = true;
+            }
             ticket = dyn_n > 0 ? int64_t(atomicAdd(p.dyn_ticket, 1)) : dyn_n;
         };
         // lane 0: the next piece to issue, or -1 when there is none
@@ -628,6 +635,9 @@ row_stats_tma_kernel(const StatsParams p) {
             if (!tickets_done && ticket >= 0 && ticket < dyn_n)
                 p.partials[decode_item<T>(p, row_start, dyn_base + ticket).partial_idx] = bad;
         }
+        // This grid completes only after the grid that zeroed the control
+        // words (the kernels after it rely on that); a no-op once waited for.
+        if (lane == 0 && !ctrl_ready) asm volatile("griddepcontrol.wait;" ::: "memory");
         // Wait until the consumers are done, then make sure no copy issued by
         // this CTA is still in flight before exiting (after a timeout).
         named_barrier_sync(2, kThreads);
@@ -711,6 +721,8 @@ row_stats_ldg_kernel(const StatsParams p) {
     __shared__ int scan_scratch[32];
     __shared__ float red[2][2 * kWarps];
     if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;");  // see the bulk-copy variant
+    // this grid completes only after the grid that zeroed the control words
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     build_row_prefix<kThreads>(p, ldg_row_start, scan_scratch);
     int64_t lo, hi;
     piece_range((int64_t)ldg_row_start[p.nB] * p.P, &lo, &hi);
