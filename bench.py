@@ -640,10 +640,11 @@ def reread_bytes(w, g_len, greedy=False) -> int:
 
 
 def launches_per_call(B: int, greedy: bool, draft_logits: bool) -> int:
-    """Kernels one spec_verify call launches: the row-statistics kernel per
-    block of up to 4096 requests, the scan kernel, and for sampling the draw
-    kernel plus (with draft logits: residual draws) the selection kernel."""
-    return math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + 1 + (0 if greedy else 1 + int(draft_logits))
+    """Kernels one spec_verify call launches: the control-word zeroing
+    kernel, the row-statistics kernel per block of up to 4096 requests, the
+    scan kernel, and for sampling the draw kernel plus (with draft logits:
+    residual draws) the selection kernel."""
+    return 1 + math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + 1 + (0 if greedy else 1 + int(draft_logits))
 
 
 def config_record(dw, cfg, steps, warmup, k1_samples, peak):
