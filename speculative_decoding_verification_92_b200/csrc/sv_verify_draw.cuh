@@ -4,9 +4,10 @@
 // The scan kernel queued one draw per sampling request: a residual draw
 // (rejection with draft logits) as P tasks, one per piece of the row pair,
 // and a bonus or one-hot draw as one task.  K2b is a persistent grid of
-// resident CTAs; CTA x takes tasks x, x + G, x + 2G, ... (residual tasks
-// first, ordered slot-major, so one draw's pieces run on P different CTAs at
-// once).  Each task stages its piece(s) in shared memory with 1-D bulk copies
+// resident CTAs; CTA x takes tasks x, x + G, x + 2G, ...; the single-piece
+// draws, whose chain is longest, take the last CTAs of the first round, and
+// the residual pieces fill the other tasks in queue order, so one draw's
+// pieces run on P different CTAs at once (TaskMap).  Each task stages its piece(s) in shared memory with 1-D bulk copies
 // (double-buffered: the next task's copies, and the queue entry of the one
 // after, are in flight while the current task is computed) and computes the
 // draw weights
@@ -334,9 +335,29 @@ __device__ __forceinline__ void pick_piece(const float* s_pw, int P, float ustar
     }
 }
 
-// The draw of task t: a queue entry, and the piece it stages first.
-__device__ __forceinline__ DrawReq task_req(const DrawParams& p, int64_t t, int64_t n_res_tasks) {
-    return t < n_res_tasks ? load_req(p.res_req + t / p.P) : load_req(p.one_req + (t - n_res_tasks));
+// Task numbering: CTA x of G runs tasks x, x + G, x + 2G, ...  The first
+// n1 = min(#single, W) single-piece draws (bonus, one-hot: the tasks with the
+// longest chain) go to the last CTAs of the first round, one each, counting
+// down from CTA W - 1 (W = min(G, #tasks)), so that no CTA runs one after
+// another task; residual pieces fill the other tasks in queue order, and any
+// further single-piece draws come last.
+struct TaskMap {
+    int n_res_tasks, ntask, W, n1;   // < B * (P + 1) <= 2^31 - 1
+    // residual piece index (>= 0: draw index / P, piece index % P), or
+    // -(1 + single-piece draw index)
+    __device__ __forceinline__ int decode(int t) const {
+        if (t < W) {
+            const int d = W - 1 - t;
+            return d < n1 ? -(1 + d) : t;
+        }
+        const int q = t - n1;
+        return q < n_res_tasks ? q : -(1 + n1 + (q - n_res_tasks));
+    }
+};
+
+// The queue entry of task code e (TaskMap::decode).
+__device__ __forceinline__ DrawReq task_req(const DrawParams& p, int e) {
+    return e >= 0 ? load_req(p.res_req + e / p.P) : load_req(p.one_req + (-e - 1));
 }
 
 template <typename T>
@@ -359,15 +380,23 @@ verify_draw_kernel(const DrawParams p) {
     // the selection kernel may be launched now; it waits for this grid
     if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
     // the scan kernel's queue (this kernel is a programmatic dependent of it);
-    // thread 0 reads its first task's entry together with the queue lengths,
-    // taking it to be a residual piece (it is, unless few draws are residual)
+    // thread 0 reads the two entries its first task can have when there are
+    // at least G tasks (residual piece x, or single-piece draw G - 1 - x)
+    // together with the queue lengths
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    DrawReq first;
-    if (tid == 0) first = load_req(p.res_req + min(int(blockIdx.x / P), p.B - 1));
+    DrawReq first, first_one;
+    if (tid == 0) {
+        first = load_req(p.res_req + min(int(blockIdx.x / P), p.B - 1));
+        first_one = load_req(p.one_req + min(int(gridDim.x - 1 - blockIdx.x), p.B - 1));
+    }
     const int nres = __ldcg(p.ctrl + 0);
     const int none = __ldcg(p.ctrl + 1);
-    const int64_t n_res_tasks = int64_t(nres) * P;
-    const int64_t ntask = n_res_tasks + none;
+    TaskMap tm;
+    tm.n_res_tasks = nres * P;
+    tm.ntask = tm.n_res_tasks + none;
+    tm.W = min(int(gridDim.x), tm.ntask);
+    tm.n1 = min(none, tm.W);
+    const int ntask = tm.ntask;
     if (blockIdx.x >= ntask) return;
     if (tid == 0) {
         mbar_init(&s_bar[0], 1);
@@ -393,9 +422,10 @@ verify_draw_kernel(const DrawParams p) {
 
     // Thread 0 only: store task t's draw r in s_req[buf] and issue the copies
     // of its first piece into buffer buf (completing on s_bar[buf]).
-    auto issue = [&](int64_t t, const DrawReq& r, int buf) {
-        const bool resid = t < n_res_tasks;
-        const int pc = resid ? static_cast<int>(t % P) : (r.mode == kBonus ? r.piece : r.x / p.PE);
+    auto issue = [&](int t, const DrawReq& r, int buf) {
+        const int e = tm.decode(t);
+        const bool resid = e >= 0;
+        const int pc = resid ? static_cast<int>(e % P) : (r.mode == kBonus ? r.piece : r.x / p.PE);
         s_req[buf] = r;
         if (r.b == p.lost_draw_b && pc == (resid ? 0 : pc)) return;  // injected fault: nothing completes the wait
         unsigned char* dst = draw_dsm + size_t(buf) * kDrawBufBytes;
@@ -424,12 +454,13 @@ verify_draw_kernel(const DrawParams p) {
     };
     // A lost draw: the request reports -2; a residual draw is also marked so
     // that the selection kernel leaves it alone.
-    auto fail_request = [&](const DrawReq& r, int64_t t) {
+    auto fail_request = [&](const DrawReq& r, int t) {
         int32_t* tok = p.out_tokens + int64_t(r.b) * (K + 1);
         for (int i = tid; i <= K; i += kDrawThreads) tok[i] = -1;
         if (tid == 0) {
             p.out_len[r.b] = -2;
-            if (t < n_res_tasks) p.res_lost[t / P] = 1;
+            const int e = tm.decode(t);
+            if (e >= 0) p.res_lost[e / P] = 1;
         }
     };
 
@@ -437,22 +468,25 @@ verify_draw_kernel(const DrawParams p) {
     // registers, loaded one iteration ahead of its use.
     DrawReq ahead;
     if (tid == 0) {
-        if (int64_t(blockIdx.x) >= n_res_tasks) first = task_req(p, blockIdx.x, n_res_tasks);
+        const int x = blockIdx.x;
+        const int e = tm.decode(x);
+        if (e < 0 && -e - 1 == int(gridDim.x) - 1 - x) first = first_one;
+        else if (!(e >= 0 && e / P == x / P)) first = task_req(p, e);
         issue(blockIdx.x, first, 0);
-        if (blockIdx.x + gridDim.x < ntask) ahead = task_req(p, blockIdx.x + gridDim.x, n_res_tasks);
+        if (blockIdx.x + gridDim.x < ntask) ahead = task_req(p, tm.decode(blockIdx.x + gridDim.x));
     }
     pend0 = true;
     int it = 0;
-    for (int64_t t = blockIdx.x; t < ntask; t += gridDim.x, ++it) {
+    for (int t = blockIdx.x; t < ntask; t += gridDim.x, ++it) {
         const int buf = it & 1;
-        const int64_t tn = t + gridDim.x;
+        const int tn = t + int(gridDim.x);
         __syncthreads();  // s_req[buf] is written; buffer buf ^ 1 is free again
         const DrawReq r = s_req[buf];
         if (tn < ntask) {
             if (tid == 0) {
                 if (failed) s_req[buf ^ 1] = ahead;   // no more copies: only the entry is passed on
                 else issue(tn, ahead, buf ^ 1);
-                if (tn + gridDim.x < ntask) ahead = task_req(p, tn + gridDim.x, n_res_tasks);
+                if (tn + gridDim.x < ntask) ahead = task_req(p, tm.decode(tn + gridDim.x));
             }
             if (!failed) {
                 if (buf) pend0 = true; else pend1 = true;
@@ -480,10 +514,11 @@ verify_draw_kernel(const DrawParams p) {
         int32_t* out_tok = p.out_tokens + int64_t(r.b) * (K + 1) + r.j;
         int pc_loaded = -1;   // piece of target row j staged in tbuf with s_seg holding its p-based segment sums
 
-        if (t < n_res_tasks) {
+        const int code = tm.decode(t);
+        if (code >= 0) {
             // residual piece: its segment sums go to the selection kernel
-            const int slot = static_cast<int>(t / P);
-            const int pc = static_cast<int>(t % P);
+            const int slot = static_cast<int>(code / P);
+            const int pc = static_cast<int>(code % P);
             piece_segments<T>(wr, tbuf, dbuf, staged_bytes(pc) / 16, vec_ok, pc * p.PE, piece_n(pc), s_seg);
             if (warp == 0) p.seg[(int64_t(slot) * P + pc) * kSegsPerPiece + lane] = s_seg[lane];
             continue;
@@ -642,7 +677,11 @@ template <typename T>
 __global__ void __launch_bounds__(kSelectThreads)
 verify_select_kernel(const SelectParams p) {
     constexpr int PV = Logit<T>::kPerVec;
-    __shared__ float s_segs[kSelectWarps][kSegsPerPiece];
+    // per warp: the segment sums of the draw's pieces as loaded (one row of
+    // 33 floats per lane, so the lanes' stores hit distinct banks), kept when
+    // every lane holds one piece (P <= 32) so that the chosen piece's sums
+    // need no second load; the zero-mass path reuses the first row
+    __shared__ float s_segs[kSelectWarps][32 * (kSegsPerPiece + 1)];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // slot < B: every load below stays inside the workspace, so the queue
@@ -674,14 +713,22 @@ verify_select_kernel(const SelectParams p) {
         float t = 0.f;
         if (k < cps && c < P) {
             const float4* s4 = reinterpret_cast<const float4*>(seg + int64_t(c) * kSegsPerPiece);
+            float* keep = &s_segs[warp][lane * (kSegsPerPiece + 1)];
 #pragma unroll
             for (int q = 0; q < kSegsPerPiece / 4; ++q) {
                 const float4 v = s4[q];
                 t += (v.x + v.y) + (v.z + v.w);
+                if (cps == 1) {
+                    keep[4 * q] = v.x;
+                    keep[4 * q + 1] = v.y;
+                    keep[4 * q + 2] = v.z;
+                    keep[4 * q + 3] = v.w;
+                }
             }
         }
         w[k] = t;
     }
+    __syncwarp();
     if (slot >= nres || lost != 0) return;
     float tot = 0.f;
 #pragma unroll
@@ -693,7 +740,7 @@ verify_select_kernel(const SelectParams p) {
     const float* segp = nullptr;
     if (tot > 0.f) {
         pstar = warp_pick<kMaxPiecesPerLane>(w, P, r.ustar * tot, &local);
-        segp = seg + int64_t(pstar) * kSegsPerPiece;
+        segp = cps == 1 ? &s_segs[warp][pstar * (kSegsPerPiece + 1)] : seg + int64_t(pstar) * kSegsPerPiece;
     } else {
         // zero residual mass (p == q numerically): draw from p_j -- the piece
         // from the partials, its segment sums computed here by the warp
