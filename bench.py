@@ -150,6 +150,22 @@ def input_bytes(w, greedy=False) -> int:
     return int(n)
 
 
+def host_copy_bytes(w, greedy=False) -> int:
+    """Bytes spec_verify_host copies to the device per call: the logit rows
+    the method reads (target rows 0..L_b, draft rows 0..L_b-1; every row when
+    no draft_lens are given), the ids, lengths and uniforms."""
+    if w.lens is None:
+        return input_bytes(w, greedy)
+    row = w.target.shape[2] * w.target.itemsize
+    L = np.clip(w.lens.astype(np.int64), 0, w.k_max)
+    n = int((L + 1).sum()) * row + w.tokens.nbytes + w.lens.nbytes
+    if w.draft is not None and not greedy:
+        n += int(L.sum()) * row
+    if not greedy:
+        n += w.uniforms.nbytes
+    return int(n)
+
+
 def workload_desc(w, cfg) -> dict:
     return {
         "workload": f"{w.name}: B={w.B} k={w.k_max} V={w.V} {w.dtype} T={w.temperature}"
@@ -743,7 +759,7 @@ def run_ours_impl(args):
         e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
         assert np.array_equal(h["out"][0].numpy(), g_len), "host entry point disagrees with device entry point"
         e2e = {"value": aggregate_value(n, positions, args.e2e_steps, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": dw.in_bytes,
+               "h2d_bytes_per_step": host_copy_bytes(w, greedy),
                "d2h_bytes_per_step": int(h["out"][0].nbytes + h["out"][1].nbytes),
                "steps": args.e2e_steps, "ms_per_step": e2e_ms / args.e2e_steps}
 

@@ -226,7 +226,11 @@ SV_API size_t spec_verify_host_staging_bytes(const sv_shape *shape, int32_t has_
 
 /* End-to-end form taking HOST buffers (same layouts as spec_verify): copies
  * the inputs into `device_staging` (cudaMemcpyAsync on `stream`), verifies,
- * and copies out_accept_len / out_tokens back to the host buffers.  The
+ * and copies out_accept_len / out_tokens back to the host buffers.  Of the
+ * logits only the rows the method reads are copied when h_draft_lens is
+ * given: target rows 0..L_b and draft rows 0..L_b-1 of each request (L_b
+ * clamped to [0, k_max]), one copy per contiguous run; the staging rows
+ * past them keep their old contents and are never read.  The
  * copies are asynchronous only when the host buffers are page-locked;
  * results are valid after the stream is synchronised.  `device_staging`
  * (spec_verify_host_staging_bytes) and `workspace` are caller-owned device

@@ -615,8 +615,49 @@ sv_status spec_verify_host(const sv_shape* shape, const void* h_target_logits, c
     auto h2d = [&](size_t off, const void* src, size_t n) {
         return n ? cudaMemcpyAsync(base + off, src, n, cudaMemcpyHostToDevice, cs) : cudaSuccess;
     };
-    cudaError_t e = h2d(h.target, h_target_logits, B * (K + 1) * st * es);
-    if (e == cudaSuccess && has_draft) e = h2d(h.draft, h_draft_logits, B * K * st * es);
+    // Logits: only the rows the kernels read -- target rows 0..L_b and draft
+    // rows 0..L_b-1 of request b, L_b clamped to [0, k_max] as the
+    // row-statistics kernel clamps it -- one copy per contiguous run (the
+    // rows of consecutive requests with L_b = k_max join up).  Without
+    // draft_lens every row is read.  Staging rows that are not copied keep
+    // whatever they held; no kernel reads them.
+    const size_t trow = st * es;
+    cudaError_t e = cudaSuccess;
+    if (!has_lens) {
+        e = h2d(h.target, h_target_logits, B * (K + 1) * trow);
+        if (e == cudaSuccess && has_draft) e = h2d(h.draft, h_draft_logits, B * K * trow);
+    } else {
+        // run-length merge of [offset, offset + n) ranges of one tensor
+        struct Run {
+            size_t off = 0, n = 0;
+        };
+        auto flush = [&](Run& r, size_t dst_base, const void* src_base) {
+            cudaError_t err = cudaSuccess;
+            if (r.n) err = h2d(dst_base + r.off, static_cast<const unsigned char*>(src_base) + r.off, r.n);
+            r = Run{};
+            return err;
+        };
+        auto add = [&](Run& r, size_t off, size_t n, size_t dst_base, const void* src_base) {
+            if (n == 0) return cudaSuccess;
+            if (r.n && r.off + r.n == off) {
+                r.n += n;
+                return cudaSuccess;
+            }
+            const cudaError_t err = flush(r, dst_base, src_base);
+            r.off = off;
+            r.n = n;
+            return err;
+        };
+        Run rt, rd;
+        for (size_t b = 0; b < B && e == cudaSuccess; ++b) {
+            const int32_t l = h_draft_lens[b];
+            const size_t L = l < 0 ? 0 : (size_t(l) > K ? K : size_t(l));
+            e = add(rt, b * (K + 1) * trow, (L + 1) * trow, h.target, h_target_logits);
+            if (e == cudaSuccess && has_draft) e = add(rd, b * K * trow, L * trow, h.draft, h_draft_logits);
+        }
+        if (e == cudaSuccess) e = flush(rt, h.target, h_target_logits);
+        if (e == cudaSuccess && has_draft) e = flush(rd, h.draft, h_draft_logits);
+    }
     if (e == cudaSuccess && K) e = h2d(h.tokens, h_draft_tokens, B * K * 4);
     if (e == cudaSuccess && has_lens) e = h2d(h.lens, h_draft_lens, B * 4);
     if (e == cudaSuccess && !greedy) e = h2d(h.uniforms, h_uniforms, B * (K + 1) * 4);

@@ -70,3 +70,29 @@ def test_host_entry_point_matches_device_entry_point():
                               torch.from_numpy(w.uniforms).pin_memory(), w.temperature)
     torch.cuda.synchronize()
     assert np.array_equal(out[0].numpy(), g_len) and np.array_equal(out[1].numpy(), g_tok)
+
+
+@pytest.mark.parametrize("greedy", [False, True])
+def test_host_entry_point_copies_only_the_rows_it_reads(greedy):
+    """Mixed draft lengths (rows past L_b are NaN in the host tensors): the
+    host entry point copies only the rows the method reads, so the staging
+    rows it skips keep what they held before -- here 0xff bytes, NaN in fp32
+    -- and the outputs still equal the device entry point's."""
+    w = workload(5)
+    g_len, g_tok = run_gpu(w, greedy=greedy)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    staging = torch.full((w.target.nbytes + w.draft.nbytes + (1 << 20),), 255, dtype=torch.uint8,
+                         device="cuda")
+    out = sv.spec_verify_host(pin(w.target), None if greedy else pin(w.draft), pin(w.tokens), pin(w.lens),
+                              None if greedy else pin(w.uniforms), w.temperature, greedy, V=w.V,
+                              staging=staging)
+    torch.cuda.synchronize()
+    assert np.array_equal(out[0].numpy(), g_len) and np.array_equal(out[1].numpy(), g_tok)
+    # the skipped rows were not written: the first padding row of a short
+    # request still holds the fill bytes
+    b = int(np.argmin(w.draft_lens))
+    L = int(w.draft_lens[b])
+    assert L < w.k_max
+    row = w.target.shape[2] * w.target.itemsize
+    off = (b * (w.k_max + 1) + L + 1) * row
+    assert bool((staging[off:off + row] == 255).all())
