@@ -196,7 +196,7 @@ def committed_traffic(kernel_variant: str, cfg: int):
     try:
         from speculative_decoding_verification_92_b200 import build as _b
         d = json.loads(TRAFFIC_FILE.read_text())
-        if d.get("source_hash") != _b.kernel_source_hash():
+        if d.get("source_hash") != _b.row_stats_source_hash():
             return None
         e = d.get("per_config", {}).get(str(cfg), {}).get(kernel_variant)
         return None if e is None else float(e["dram_bytes_per_launch"])

@@ -48,9 +48,10 @@
  * spec_verify_ex and spec_verify_stats is DEVICE memory owned by the caller
  * (spec_verify_host takes host buffers, see there).  The library allocates
  * nothing.  Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL
- * = legacy default stream) as three kernels -- row statistics, the acceptance
- * scan and (sampling only) the final draw; results are valid once the stream
- * has reached the call's end.  The workspace (per-piece row statistics and
+ * = legacy default stream) as a chain of kernels -- a control-word reset, row
+ * statistics, the acceptance scan and (sampling only) the final draw, plus
+ * the selection of residual draws when draft logits are given; results are
+ * valid once the stream has reached the call's end.  The workspace (per-piece row statistics and
  * the queue of draws) needs no initialisation and holds nothing between
  * calls; two calls that run concurrently need separate workspaces.
  * The host keeps one small per-device cache of SM count and kernel

@@ -53,6 +53,22 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
+def row_stats_source_hash() -> str:
+    """Hash of what the row-statistics kernel is built and launched from: its
+    header, the shared device helpers and the launch function in
+    spec_verify.cu.  DRAM counters taken on that kernel stay valid while this
+    is unchanged (edits to the other kernels do not touch them)."""
+    h = hashlib.sha256()
+    for s in (CSRC / "sv_row_stats.cuh", CSRC / "sv_common.cuh"):
+        h.update(s.name.encode())
+        h.update(s.read_bytes())
+    cu = (CSRC / "spec_verify.cu").read_text()
+    start = cu.index("cudaError_t launch_stats(")
+    h.update(cu[start:cu.index("\n}\n", start)].encode())
+    h.update(" ".join(ARCH).encode())
+    return h.hexdigest()
+
+
 def source_hash() -> str:
     h = hashlib.sha256()
     for s in sources():
