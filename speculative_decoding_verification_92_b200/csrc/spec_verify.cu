@@ -117,9 +117,19 @@ cudaError_t device_info(DeviceInfo** out) {
     return cudaSuccess;
 }
 
+// Every kernel of a call asks for the largest shared-memory carveout, so
+// consecutive kernels find the SMs in the same L1 / shared-memory split and
+// a dependent grid's CTAs can move in while the previous grid drains.
+template <typename Kernel>
+cudaError_t prefer_smem(Kernel k) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
 // Opt a kernel into `bytes` of dynamic shared memory (idempotent per device).
 template <typename Kernel>
 cudaError_t allow_smem(Kernel k, size_t bytes) {
+    const cudaError_t e = prefer_smem(k);
+    if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
@@ -192,11 +202,14 @@ struct NvtxRange {
     ~NvtxRange() { nvtxRangePop(); }
 };
 
-// Zeroes the control words.  It lets the row-statistics kernel launch at
-// once (as its programmatic dependent); that kernel waits for this grid only
-// before its first ticket, so its prologue and first copies overlap this
-// launch.
+// Zeroes the control words.  It is itself a programmatic dependent of
+// whatever precedes the call on the stream (the previous call's last kernel
+// lets it in early), so it first waits for that work to complete; then it
+// lets the row-statistics kernel launch (as its programmatic dependent: that
+// kernel waits for this grid only before its first ticket, so its prologue
+// and first copies overlap this one) and zeroes the words.
 __global__ void zero_ctrl_kernel(int32_t* ctrl, int n) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     for (int i = threadIdx.x; i < n; i += blockDim.x) ctrl[i] = 0;
 }
@@ -301,6 +314,7 @@ cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, const S
     // residual draws need draft logits: with one-hot q the queue holds none
     if (cp.draft == nullptr) return cudaSuccess;
     auto k = verify_select_kernel<T>;
+    if (cudaError_t e = prefer_smem(k); e != cudaSuccess) return e;
     cfg.gridDim = dim3(static_cast<unsigned>((int64_t(B) + kSelectWarps - 1) / kSelectWarps));
     cfg.blockDim = dim3(kSelectThreads);
     cfg.dynamicSmemBytes = 0;
@@ -395,9 +409,21 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     const int lost = a.opts ? a.opts->lost_copy_request : 0;
     sp.lost_copy_partial = lost > 0 ? int64_t(lost - 1) * (2 * s.k_max + 1) * plan.P : -1;
 
-    zero_ctrl_kernel<<<1, 32, 0, a.stream>>>(ctrl, static_cast<int>(ctrl_ints(s)));
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = prefer_smem(zero_ctrl_kernel);
     if (e != cudaSuccess) return SV_ECUDA;
+    {
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1);
+        cfg.blockDim = dim3(32);
+        cfg.stream = a.stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&cfg, zero_ctrl_kernel, ctrl, static_cast<int>(ctrl_ints(s)))) != cudaSuccess)
+            return SV_ECUDA;
+    }
     if (a.opts && a.opts->event_stats_begin)
         if ((e = cudaEventRecord(static_cast<cudaEvent_t>(a.opts->event_stats_begin), a.stream)) != cudaSuccess)
             return SV_ECUDA;

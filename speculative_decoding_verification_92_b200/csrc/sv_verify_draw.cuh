@@ -683,6 +683,8 @@ verify_select_kernel(const SelectParams p) {
     // need no second load; the zero-mass path reuses the first row
     __shared__ float s_segs[kSelectWarps][32 * (kSegsPerPiece + 1)];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the next call's first kernel may be launched now; it waits for this grid
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // slot < B: every load below stays inside the workspace, so the queue
     // length, the loss mark, the entry and the segment sums are read at once
