@@ -544,10 +544,10 @@ def pin_accept_sim_matches_verify_and_monte_carlo(orc):
 
 
 # --------------------------------------------------------------------------
-# Near-tie flags (the benchmark spec: the generator and oracle flag positions where
-# |u - min(1, p/q)| or the residual-CDF margin is below 1e-5) and the two
-# fallback branches of the rule's readings (no step above u*W: the largest
-# positive-weight token; zero residual mass: draw from p_j).
+# Near-tie flags (the oracle flags a request whose |u - min(1, p/q)| at an
+# examined position, or whose residual-CDF margin relative to W, is below
+# 1e-5) and the two fallback branches of the rule's readings (no step above
+# u*W: the largest positive-weight token; zero residual mass: draw from p_j).
 
 
 def _flags(orc, target, draft, tokens, u, T=1.0):
