@@ -1,6 +1,6 @@
 """GPU edge cases against the oracle: every row-statistics kernel, ragged
 vocabulary tails, tiny and single-token vocabularies, empty drafts, padded
-and misaligned rows, temperatures, greedy ties across chunk boundaries,
+and misaligned rows, temperatures, greedy ties across piece boundaries,
 extreme uniforms, invalid ids / lengths, large batches split over several
 launches, the largest vocabulary and draft length, and closed forms of the
 rule."""
@@ -112,10 +112,10 @@ def test_extreme_uniforms(u):
     compare(w, g_len, g_tok, o, diag=o)
 
 
-def test_greedy_ties_across_chunk_boundary():
+def test_greedy_ties_across_piece_boundaries():
     V = 151936
     w = make_workload(B=3, k_max=2, V=V, dtype=BF16, seed=14, draft_mode="ids")
-    CE = 24576  # chunk length for this vocabulary: 3 stages of 16 KiB
+    CE = 3 * 8192  # three bf16 pieces of 16 KiB: CE - 1 and CE sit in pieces 2 and 3
     for b in range(3):
         for i in range(3):
             row = np.zeros(V, np.float32)
@@ -149,11 +149,11 @@ def test_invalid_requests_are_reported_not_read():
 
 @pytest.mark.parametrize("dtype", [F32, BF16])
 def test_largest_vocabulary(dtype):
-    # V = MAX_V: 8 chunks of 192 KiB (fp32, beyond the ring draw: the segment
-    # draw with 16-byte loads) or of 96 KiB (bf16, the ring draw)
+    # V = MAX_V: 96 pieces of 16 KiB per fp32 row (48 per bf16 row), so the
+    # selection sums more than 32 pieces per draw
     # heavy-tailed logits (sigma 4): the mass sits on a few hundred ids spread
     # over the whole row, so most draws are far from a near-tie and compare
-    # exactly, while the chunk and segment sums still span every chunk
+    # exactly, while the piece and segment sums still span every piece
     w = make_workload(B=6, k_max=2, V=sv.MAX_V, dtype=dtype, seed=61, z_sigma=4.0, boost=0.0,
                       draft_noise=0.5, lens=[2, 1, 0, 2, 2, 1])
     o = check(w)

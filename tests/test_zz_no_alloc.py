@@ -43,7 +43,7 @@ def call_static(w, d, greedy=False):
 
 
 def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
-    w1 = make_config(2)                                   # 64 x 17 rows x 7 chunks of partials
+    w1 = make_config(2)                                   # 64 x 17 rows x 19 pieces of partials
     w2 = make_workload(B=33, k_max=12, V=20000, dtype="f32", seed=5, boost=4.0, draft_noise=0.3,
                        lens_choices=(0, 4, 12), lens_probs=(0.4, 0.3, 0.3))
     assert sv.workspace_bytes(w1.B, w1.k_max, w1.V, sv.BF16) <= SCRATCH_BYTES
@@ -60,7 +60,7 @@ def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
 
 
 def test_static_scratch_rejects_problems_larger_than_its_array():
-    w = make_workload(B=600, k_max=16, V=64, dtype="f32", seed=6)   # fits: 600 * 33 rows * 1 chunk * 8 B
+    w = make_workload(B=600, k_max=16, V=64, dtype="f32", seed=6)   # fits: 600 * 33 rows * 1 piece * 8 B + draw queue
     assert sv.workspace_bytes(w.B, w.k_max, w.V, sv.F32) <= SCRATCH_BYTES
     lib = sv.library()
     big = _Shape(4096, 64, 151936, sv.BF16, 0)                      # partials far beyond 1 MiB
