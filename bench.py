@@ -655,12 +655,26 @@ def reread_bytes(w, g_len, greedy=False) -> int:
     return int((1 + resid.astype(np.int64)).sum()) * w.V * w.esize
 
 
-def launches_per_call(B: int, greedy: bool, draft_logits: bool) -> int:
+def draw_path_of(sv, w, greedy) -> str:
+    """The draw path the library's AUTO choice takes for this workload
+    ("cluster" or "queue"; greedy calls make no draw)."""
+    if greedy:
+        return "none"
+    dt = sv.BF16 if w.dtype == "bf16" else sv.F32
+    path = sv.auto_draw_path(w.B, w.k_max, w.V, dt, w.target.shape[2])
+    return "cluster" if path == sv.DrawPath.CLUSTER else "queue"
+
+
+def launches_per_call(B: int, path: str, draft_logits: bool) -> int:
     """Kernels one spec_verify call launches: the control-word zeroing
-    kernel, the row-statistics kernel per block of up to 4096 requests, the
-    scan kernel, and for sampling the draw kernel plus (with draft logits:
+    kernel, the row-statistics kernel per block of up to 4096 requests, then
+    the scan kernel alone (greedy), the cluster kernel (scan and draw, small
+    batches), or the scan kernel, the draw kernel and (with draft logits:
     residual draws) the selection kernel."""
-    return 1 + math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH) + 1 + (0 if greedy else 1 + int(draft_logits))
+    n = 1 + math.ceil(B / MAX_REQUESTS_PER_STATS_LAUNCH)
+    if path in ("none", "cluster"):
+        return n + 1
+    return n + 2 + int(draft_logits)
 
 
 def config_record(dw, cfg, steps, warmup, k1_samples, peak):
@@ -684,7 +698,7 @@ def config_record(dw, cfg, steps, warmup, k1_samples, peak):
         "k1_gbs_median": alg / (k1_med / 1e3) / 1e9, "k1_frac_median": alg / (k1_med / 1e3) / 1e9 / peak,
         "k1_frac_mean": alg / (k1_mean / 1e3) / 1e9 / peak,
         "accept_rate": float(g_len.sum() / max(1, w.positions)), "mean_accept_len": float(g_len.mean()),
-        "parity": parity,
+        "draw_path": draw_path_of(dw.sv, w, dw.greedy), "parity": parity,
     }
 
 
@@ -789,7 +803,8 @@ def run_ours_impl(args):
     cfgd = workload_desc(w, args.config)
     cfgd.update({"parallelism": f"replicas{n}" if n > 1 else "single",
                  "sharding": "each rank verifies its own batch; no data-path collective",
-                 "l2": dw.l2_note, "stats_kernel": variant, "greedy": greedy})
+                 "l2": dw.l2_note, "stats_kernel": variant, "greedy": greedy,
+                 "draw_path": draw_path_of(sv, w, greedy)})
     dw.release()
 
     # ---------------- the other workloads (rank 0, N = 1) ----------------
@@ -817,7 +832,7 @@ def run_ours_impl(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": K, "warmup": W,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic", "config": cfgd,
-            "e2e": e2e, "gpu_launches": K * launches_per_call(w.B, greedy, w.draft is not None), "roofline": roofline,
+            "e2e": e2e, "gpu_launches": K * launches_per_call(w.B, draw_path_of(sv, w, greedy), w.draft is not None), "roofline": roofline,
             "cpu_baseline": cpu, "clocks": clocks.summary(),
             "hbm_gbs": alg / (ms_per_step / 1e3) / 1e9,
             "accept_rate": accept_rate, "mean_accept_len": float(g_len.mean()),

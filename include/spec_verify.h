@@ -87,7 +87,7 @@ extern "C" {
 #define SV_API
 #endif
 
-#define SV_ABI_VERSION 2
+#define SV_ABI_VERSION 3
 #define SV_MAX_K 1024      /* largest supported k_max */
 #define SV_MAX_V 393216    /* largest supported vocabulary (96 pieces of 16 KiB in fp32) */
 
@@ -143,8 +143,20 @@ typedef struct {
      * and the context stays usable.  No effect on calls without a draw
      * (greedy, statistics). */
     int32_t lost_draw_request;
-    int32_t reserved[6];       /* must be zero */
+    /* How a sampling call makes its final draws (sv_draw_path).  AUTO: one
+     * thread-block cluster per request when the batch's clusters fit on the
+     * GPU at once (small batches: the scan and the draw in one kernel), else
+     * the scan kernel, the draw kernel over a queue of pieces and the
+     * residual selection kernel.  The outputs are the same either way. */
+    int32_t draw_path;
+    int32_t reserved[5];       /* must be zero */
 } sv_options;
+
+typedef enum {
+    SV_DRAW_AUTO = 0,
+    SV_DRAW_QUEUE = 1,    /* scan kernel, draw kernel, selection kernel */
+    SV_DRAW_CLUSTER = 2   /* one cluster of up to 8 CTAs per request */
+} sv_draw_path;
 
 /* Bytes of device workspace spec_verify / spec_verify_stats need for this
  * shape (0 on an invalid shape). */
@@ -248,6 +260,11 @@ SV_API sv_status spec_verify_host(const sv_shape *shape, const void *h_target_lo
 
 /* Static description of a status code. */
 SV_API const char *spec_verify_status_string(sv_status status);
+
+/* The draw path (sv_draw_path) that SV_DRAW_AUTO takes for a sampling call
+ * of this shape on the current device: SV_DRAW_CLUSTER or SV_DRAW_QUEUE; -1
+ * on an invalid shape or a CUDA error.  No work is enqueued. */
+SV_API int32_t spec_verify_auto_draw_path(const sv_shape *shape);
 
 /* SV_ABI_VERSION of the built library. */
 SV_API int32_t spec_verify_abi_version(void);

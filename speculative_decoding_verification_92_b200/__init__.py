@@ -25,7 +25,7 @@ from pathlib import Path
 __all__ = [
     "Status", "StatsKernel", "SpecVerifyError", "library", "workspace_bytes",
     "spec_verify", "spec_verify_stats", "spec_verify_accept_sim", "spec_verify_host", "host_staging_bytes",
-    "abi_version", "F32", "BF16", "MAX_K", "MAX_V",
+    "abi_version", "auto_draw_path", "DrawPath", "F32", "BF16", "MAX_K", "MAX_V",
 ]
 
 F32 = 0
@@ -49,6 +49,12 @@ class StatsKernel(enum.IntEnum):
     SCALAR = 3
 
 
+class DrawPath(enum.IntEnum):
+    AUTO = 0
+    QUEUE = 1     # scan kernel, draw kernel over a queue of pieces, selection kernel
+    CLUSTER = 2   # one thread-block cluster per request: scan and draw in one kernel
+
+
 class SpecVerifyError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = Status(status)
@@ -64,7 +70,7 @@ class _Options(ctypes.Structure):
     _fields_ = [("stats_kernel", ctypes.c_int32), ("wait_timeout_us", ctypes.c_int32),
                 ("event_stats_begin", ctypes.c_void_p), ("event_stats_end", ctypes.c_void_p),
                 ("lost_copy_request", ctypes.c_int32), ("lost_draw_request", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("draw_path", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
 
 
 _LIB = None
@@ -85,6 +91,7 @@ _SIGNATURES = {
                                 _VP, _SZ, _VP]),
     "spec_verify_status_string": (ctypes.c_char_p, [_I32]),
     "spec_verify_abi_version": (_I32, []),
+    "spec_verify_auto_draw_path": (_I32, [ctypes.POINTER(_Shape)]),
     "spec_verify_static_scratch": (_I32, [ctypes.POINTER(_Shape), _VP, _VP, _VP, _VP, _VP, _F32, _I32, _VP, _VP,
                                           _VP]),
 }
@@ -120,6 +127,16 @@ def library() -> ctypes.CDLL:
 
 def abi_version() -> int:
     return int(library().spec_verify_abi_version())
+
+
+def auto_draw_path(B: int, k_max: int, V: int, dtype: int, row_stride: int = 0) -> "DrawPath":
+    """The draw path DrawPath.AUTO takes for a sampling call of this shape on
+    the current device (needs a GPU)."""
+    shape = _shape(B, k_max, V, dtype, row_stride or V)
+    r = int(library().spec_verify_auto_draw_path(ctypes.byref(shape)))
+    if r < 0:
+        raise SpecVerifyError(int(Status.EINVAL), "spec_verify_auto_draw_path")
+    return DrawPath(r)
 
 
 def _check(status: int, what: str):
@@ -192,9 +209,10 @@ def _stream_handle(stream):
 
 
 def _options(stats_kernel=StatsKernel.AUTO, wait_timeout_us=0, events=None, lost_copy_request=0,
-             lost_draw_request=0):
+             lost_draw_request=0, draw_path=0):
     o = _Options()
     o.stats_kernel = int(stats_kernel)
+    o.draw_path = int(draw_path)
     o.wait_timeout_us = int(wait_timeout_us)
     o.lost_copy_request = int(lost_copy_request)
     o.lost_draw_request = int(lost_draw_request)
@@ -219,14 +237,15 @@ def _logit_shape(target, draft, V):
 
 def spec_verify(target, draft, tokens, lens, uniforms, temperature=1.0, greedy=False, *, V=None,
                 out=None, workspace=None, stream=None, stats_kernel=StatsKernel.AUTO,
-                wait_timeout_us=0, events=None, lost_copy_request=0, lost_draw_request=0):
+                wait_timeout_us=0, events=None, lost_copy_request=0, lost_draw_request=0, draw_path=0):
     """Verify one batch on the GPU.  Returns ``(accept_len [B] int32,
     tokens [B, k_max+1] int32)`` (device tensors, valid once ``stream`` has
     run).  ``events=(begin, end)`` (torch.cuda.Event, already created)
     brackets the row-statistics kernel.  ``lost_copy_request`` and
     ``lost_draw_request`` are the test-only fault injections of
     ``sv_options`` (1 + the request whose first bulk copy in the
-    row-statistics / draw kernel is never issued; 0 = off)."""
+    row-statistics / draw kernel is never issued; 0 = off).  ``draw_path``
+    picks how the final draws are made (DrawPath; AUTO by default)."""
     torch = _torch()
     B, k_max, V, dt, row_stride = _logit_shape(target, draft, V)
     dev = target.device
@@ -243,7 +262,7 @@ def spec_verify(target, draft, tokens, lens, uniforms, temperature=1.0, greedy=F
     if workspace is None:
         workspace = torch.empty(max(lib.spec_verify_workspace_bytes(ctypes.byref(shape)), 256),
                                 dtype=torch.uint8, device=dev)
-    opts = _options(stats_kernel, wait_timeout_us, events, lost_copy_request, lost_draw_request)
+    opts = _options(stats_kernel, wait_timeout_us, events, lost_copy_request, lost_draw_request, draw_path)
     st = lib.spec_verify_ex(
         ctypes.byref(shape), _dev_ptr(target, what="target"), _dev_ptr(draft, what="draft"),
         _dev_ptr(tokens, torch.int32, "draft_tokens"), _dev_ptr(lens, torch.int32, "draft_lens"),

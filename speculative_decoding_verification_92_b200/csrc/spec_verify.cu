@@ -5,7 +5,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
@@ -15,6 +17,7 @@
 #include "sv_row_stats.cuh"
 #include "sv_verify_scan.cuh"
 #include "sv_verify_draw.cuh"
+#include "sv_verify_cluster.cuh"
 
 namespace sv {
 namespace {
@@ -117,20 +120,60 @@ cudaError_t device_info(DeviceInfo** out) {
     return cudaSuccess;
 }
 
-// Every kernel of a call asks for the largest shared-memory carveout, so
-// consecutive kernels find the SMs in the same L1 / shared-memory split and
-// a dependent grid's CTAs can move in while the previous grid drains.
-template <typename Kernel>
-cudaError_t prefer_smem(Kernel k) {
-    return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-}
+// Launch setup of a kernel, done once per context and kernel (later calls
+// find it in small tables): the kernel asks for the largest shared-memory
+// carveout -- so consecutive kernels find the SMs in the same L1 /
+// shared-memory split and a dependent grid's CTAs can move in while the
+// previous grid drains -- and opts into the largest dynamic shared memory
+// any call has needed so far (the attribute only grows, so every earlier
+// size still launches); *per_sm (if given) receives the resident blocks per
+// SM for this size and block size.  Without a context id (the driver cannot
+// tell) nothing is cached.
+struct SetupKey {
+    unsigned long long ctx;
+    const void* kernel;
+    size_t smem;
+    int threads;
+    bool operator<(const SetupKey& o) const {
+        return std::tie(ctx, kernel, smem, threads) < std::tie(o.ctx, o.kernel, o.smem, o.threads);
+    }
+};
+std::map<std::pair<unsigned long long, const void*>, size_t> g_smem_set;  // largest opt-in set per kernel
+std::map<SetupKey, int> g_resident;                                        // resident blocks per SM
+std::mutex g_setup_mutex;
+constexpr size_t kMaxSetupEntries = 4096;
 
-// Opt a kernel into `bytes` of dynamic shared memory (idempotent per device).
 template <typename Kernel>
-cudaError_t allow_smem(Kernel k, size_t bytes) {
-    const cudaError_t e = prefer_smem(k);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+cudaError_t kernel_setup(Kernel k, size_t smem, int threads, int* per_sm) {
+    const SetupKey key{current_context_id(), reinterpret_cast<const void*>(k), smem, threads};
+    const auto kk = std::make_pair(key.ctx, key.kernel);
+    bool attrs_ok = false;
+    int n = -1;
+    if (key.ctx != 0) {
+        std::lock_guard<std::mutex> lock(g_setup_mutex);
+        const auto a = g_smem_set.find(kk);
+        attrs_ok = a != g_smem_set.end() && a->second >= smem;
+        const auto it = g_resident.find(key);
+        if (it != g_resident.end()) n = it->second;
+    }
+    cudaError_t e = cudaSuccess;
+    if (!attrs_ok) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    if (n < 0 && (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem)) != cudaSuccess) return e;
+    if (key.ctx != 0) {
+        std::lock_guard<std::mutex> lock(g_setup_mutex);
+        if (g_resident.size() >= kMaxSetupEntries) g_resident.clear();
+        g_resident[key] = n;
+        if (!attrs_ok) {
+            size_t& m = g_smem_set[kk];
+            if (smem > m) m = smem;
+        }
+    }
+    if (per_sm) *per_sm = n;
+    return cudaSuccess;
 }
 
 struct Plan {
@@ -234,13 +277,10 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
         if (variant == SV_STATS_TMA) {
             auto k = row_stats_tma_kernel<T, kGreedy, kTmaConsumerWarps, kTmaStages>;
             const size_t smem = TmaSmem<kTmaConsumerWarps, kTmaStages>::bytes(prm.nB);
-            if ((e = allow_smem(k, smem)) != cudaSuccess) return e;
             // one wave of resident CTAs (a long request list can make the
             // row prefix in shared memory lower the occupancy)
             int per_sm = 0;
-            if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, (kTmaConsumerWarps + 1) * 32, smem)) !=
-                cudaSuccess)
-                return e;
+            if ((e = kernel_setup(k, smem, (kTmaConsumerWarps + 1) * 32, &per_sm)) != cudaSuccess) return e;
             per_sm = per_sm < 1 ? 1 : (per_sm > TmaCtasPerSm<T>::value ? TmaCtasPerSm<T>::value : per_sm);
             const int64_t cap = int64_t(dev.sm_count) * per_sm;
             const int64_t grid = items_upper < cap ? items_upper : cap;
@@ -252,10 +292,8 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
             auto k = variant == SV_STATS_VEC16 ? row_stats_ldg_kernel<T, kGreedy, true, kLdgThreads>
                                                : row_stats_ldg_kernel<T, kGreedy, false, kLdgThreads>;
             const size_t smem = 4 * size_t(prm.nB + 1);
-            if ((e = allow_smem(k, smem)) != cudaSuccess) return e;
             int per_sm = 0;
-            if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kLdgThreads, smem)) != cudaSuccess)
-                return e;
+            if ((e = kernel_setup(k, smem, kLdgThreads, &per_sm)) != cudaSuccess) return e;
             if (per_sm < 1) per_sm = 1;
             const int64_t cap = int64_t(dev.sm_count) * per_sm;
             const int64_t grid = items_upper < cap ? items_upper : cap;
@@ -272,9 +310,65 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
 // K2a (one CTA per request), then for sampling K2b (persistent, one wave) and,
 // with draft logits, K2c (one warp per possible residual draw), each a
 // programmatic dependent of the kernel before it.
+// AUTO's choice: the cluster path when the batch's CTAs fit in half of one
+// resident wave of the cluster kernel (clusters are placed whole, inside one
+// GPC), so every request's cluster starts at once.
+template <typename T>
+cudaError_t cluster_fits(int B, int k_max, int P, const DeviceInfo& dev, bool* fits) {
+    int per_sm = 0;
+    const cudaError_t e = kernel_setup(verify_cluster_kernel<T>, cluster_smem_bytes(k_max, P), kScanThreads, &per_sm);
+    if (e != cudaSuccess) return e;
+    *fits = int64_t(B) * cluster_ctas(P) * 2 <= int64_t(per_sm) * dev.sm_count;
+    return cudaSuccess;
+}
+
+// The cluster path for a sampling call: one cluster of cluster_ctas(P) CTAs
+// per request, as a programmatic dependent of the row statistics.  AUTO
+// takes it when the batch's CTAs fit in half of one resident wave (clusters
+// are placed whole, inside one GPC).
+template <typename T>
+cudaError_t launch_cluster(const ScanParams& sp, const DrawParams& dp, int B, int path, const DeviceInfo& dev,
+                           cudaStream_t st, bool* launched) {
+    *launched = false;
+    if (path == SV_DRAW_QUEUE) return cudaSuccess;
+    auto k = verify_cluster_kernel<T>;
+    const int C = cluster_ctas(dp.P);
+    const size_t smem = cluster_smem_bytes(dp.k_max, dp.P);
+    if (path == SV_DRAW_AUTO) {
+        bool fits = false;
+        const cudaError_t e = cluster_fits<T>(B, dp.k_max, dp.P, dev, &fits);
+        if (e != cudaSuccess || !fits) return e;
+    } else if (const cudaError_t e = kernel_setup(k, smem, kScanThreads, nullptr); e != cudaSuccess) {
+        return e;
+    }
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(C);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(int64_t(B) * C));
+    cfg.blockDim = dim3(kScanThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k, sp, dp);
+    if (e != cudaSuccess) return e;
+    *launched = true;
+    return cudaSuccess;
+}
+
 template <typename T>
 cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, const SelectParams& cp, int B, bool draw,
-                             const DeviceInfo& dev, cudaStream_t st) {
+                             int path, const DeviceInfo& dev, cudaStream_t st) {
+    if (draw) {
+        bool launched = false;
+        const cudaError_t e = launch_cluster<T>(sp, dp, B, path, dev, st, &launched);
+        if (e != cudaSuccess || launched) return e;
+    }
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -285,7 +379,7 @@ cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, const S
     {
         auto k = verify_scan_kernel<T>;
         const size_t smem = scan_smem_bytes(sp.k_max, sp.P);
-        cudaError_t e = allow_smem(k, smem);
+        cudaError_t e = kernel_setup(k, smem, kScanThreads, nullptr);
         if (e != cudaSuccess) return e;
         cfg.gridDim = dim3(static_cast<unsigned>(B));
         cfg.blockDim = dim3(kScanThreads);
@@ -295,14 +389,11 @@ cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, const S
     if (!draw) return cudaSuccess;
     {
         auto k = verify_draw_kernel<T>;
-        cudaError_t e = allow_smem(k, kDrawSmemBytes);
-        if (e != cudaSuccess) return e;
         // persistent: at most one wave of resident CTAs, and no more than the
         // largest possible number of tasks
         int per_sm = 0;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kDrawThreads, kDrawSmemBytes)) !=
-            cudaSuccess)
-            return e;
+        cudaError_t e = kernel_setup(k, kDrawSmemBytes, kDrawThreads, &per_sm);
+        if (e != cudaSuccess) return e;
         per_sm = per_sm < 1 ? 1 : (per_sm > kDrawCtasPerSm ? kDrawCtasPerSm : per_sm);
         const int64_t cap = int64_t(dev.sm_count) * per_sm;
         const int64_t max_tasks = int64_t(B) * (dp.P + 1);
@@ -314,7 +405,7 @@ cudaError_t launch_scan_draw(const ScanParams& sp, const DrawParams& dp, const S
     // residual draws need draft logits: with one-hot q the queue holds none
     if (cp.draft == nullptr) return cudaSuccess;
     auto k = verify_select_kernel<T>;
-    if (cudaError_t e = prefer_smem(k); e != cudaSuccess) return e;
+    if (cudaError_t e = kernel_setup(k, 0, kSelectThreads, nullptr); e != cudaSuccess) return e;
     cfg.gridDim = dim3(static_cast<unsigned>((int64_t(B) + kSelectWarps - 1) / kSelectWarps));
     cfg.blockDim = dim3(kSelectThreads);
     cfg.dynamicSmemBytes = 0;
@@ -409,7 +500,7 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     const int lost = a.opts ? a.opts->lost_copy_request : 0;
     sp.lost_copy_partial = lost > 0 ? int64_t(lost - 1) * (2 * s.k_max + 1) * plan.P : -1;
 
-    cudaError_t e = prefer_smem(zero_ctrl_kernel);
+    cudaError_t e = kernel_setup(zero_ctrl_kernel, 0, 32, nullptr);
     if (e != cudaSuccess) return SV_ECUDA;
     {
         cudaLaunchAttribute attr[1];
@@ -479,7 +570,8 @@ sv_status run_typed(const Call& a, const Plan& plan, const DeviceInfo& dev, int 
     xp.rows_aligned = dp.rows_aligned;
     {
         NvtxRange range("spec_verify: scan, draw, selection");
-        e = launch_scan_draw<T>(cp, dp, xp, s.B, !greedy && !a.stats_only, dev, a.stream);
+        e = launch_scan_draw<T>(cp, dp, xp, s.B, !greedy && !a.stats_only, a.opts ? a.opts->draw_path : SV_DRAW_AUTO,
+                                dev, a.stream);
     }
     return e == cudaSuccess ? SV_OK : SV_ECUDA;
 }
@@ -489,8 +581,9 @@ sv_status run(const Call& a) {
     if (!shape_ok(a.shape, &why)) return why;
     const sv_shape& s = *a.shape;
     if (a.opts) {
-        for (int i = 0; i < 6; ++i)
+        for (int i = 0; i < 5; ++i)
             if (a.opts->reserved[i] != 0) return SV_EINVAL;
+        if (a.opts->draw_path < SV_DRAW_AUTO || a.opts->draw_path > SV_DRAW_CLUSTER) return SV_EINVAL;
         if (a.opts->lost_copy_request < 0 || a.opts->lost_copy_request > s.B) return SV_EINVAL;
         if (a.opts->lost_draw_request < 0 || a.opts->lost_draw_request > s.B) return SV_EINVAL;
         if (a.opts->stats_kernel < SV_STATS_AUTO || a.opts->stats_kernel > SV_STATS_SCALAR) return SV_EINVAL;
@@ -726,5 +819,19 @@ const char* spec_verify_status_string(sv_status status) {
 }
 
 int32_t spec_verify_abi_version(void) { return SV_ABI_VERSION; }
+
+int32_t spec_verify_auto_draw_path(const sv_shape* shape) {
+    sv_status why;
+    if (!sv::shape_ok(shape, &why)) return -1;
+    sv::DeviceInfo* dev = nullptr;
+    if (sv::device_info(&dev) != cudaSuccess) return -1;
+    const sv::Plan plan = sv::make_plan(*shape);
+    bool fits = false;
+    const cudaError_t e = shape->dtype == SV_BF16
+                              ? sv::cluster_fits<sv::bf16_bits>(shape->B, shape->k_max, plan.P, *dev, &fits)
+                              : sv::cluster_fits<float>(shape->B, shape->k_max, plan.P, *dev, &fits);
+    if (e != cudaSuccess) return -1;
+    return fits ? SV_DRAW_CLUSTER : SV_DRAW_QUEUE;
+}
 
 }  // extern "C"

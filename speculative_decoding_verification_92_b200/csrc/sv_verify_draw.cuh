@@ -647,6 +647,86 @@ verify_draw_kernel(const DrawParams p) {
     }
 }
 
+// One warp: the residual draw r from its piece totals w (lane l holding
+// pieces [l*cps, l*cps + cps)): the piece and the segment holding u*W, then
+// the vector and the element, re-reading that segment of both rows
+// (seg_of(c) returns piece c's 32 segment sums where the whole warp can read
+// them).  Zero residual mass (p == q numerically) draws from p_j instead:
+// the piece from the partials, its segment sums computed here by the warp
+// into s_tmp (32 floats).  Returns the token, or -1 when no positive weight
+// is found (not reached with finite logits).  Used by the cluster kernel;
+// the selection kernel below takes the same steps inline, interleaved with
+// its loads (0.7 us per step faster on the largest workload than calling
+// this function).  Their picks are identical.
+template <typename T, typename Params, typename SegOf>
+__device__ __forceinline__ int select_residual_warp(const Params& p, const DrawReq& r,
+                                                    const float (&w)[kMaxPiecesPerLane], SegOf seg_of,
+                                                    float* s_tmp) {
+    constexpr int PV = Logit<T>::kPerVec;
+    const int lane = threadIdx.x & 31;
+    const int K = p.k_max;
+    const int P = p.P;
+    const int64_t esz = Logit<T>::kSize;
+    const bool vec_ok = p.rows_aligned != 0;
+    const int cps = (P + 31) / 32;
+    WeightRow wr;
+    wr.trow = p.target + (int64_t(r.b) * (K + 1) + r.j) * p.row_stride * esz;
+    wr.drow = p.draft + (int64_t(r.b) * K + r.j) * p.row_stride * esz;
+    wr.scale = p.scale;
+    wr.lse_p = r.lse_p;
+    wr.lse_q = r.lse_q;
+    wr.mode = kResidual;
+    wr.zero_at = -1;
+    float tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMaxPiecesPerLane; ++k) tot += w[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    float local = INFINITY;
+    int pstar = -1;
+    const float* segp = nullptr;
+    if (tot > 0.f) {
+        pstar = warp_pick<kMaxPiecesPerLane>(w, P, r.ustar * tot, &local);
+        if (pstar >= 0) segp = seg_of(pstar);
+    } else {
+        wr.mode = kBonus;
+        wr.drow = nullptr;
+        const float2* part_j = p.partials + (int64_t(r.b) * (2 * K + 1) + r.j) * P;
+        float pw[kMaxPiecesPerLane];
+        float ptot = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxPiecesPerLane; ++k) {
+            const int c = lane * cps + k;
+            pw[k] = 0.f;
+            if (k < cps && c < P) {
+                const float2 pp = part_j[c];
+                pw[k] = pp.y * exp2f(pp.x - wr.lse_p);
+            }
+            ptot += pw[k];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ptot += __shfl_xor_sync(0xffffffffu, ptot, o);
+        if (ptot > 0.f) pstar = warp_pick<kMaxPiecesPerLane>(pw, P, r.ustar * ptot, &local);
+        if (pstar >= 0) {
+            const int e0 = pstar * p.PE, n = min(p.V - e0, p.PE);
+            const int nvec = (n + PV - 1) / PV;
+            for (int sg = 0; sg < kSegsPerPiece; ++sg) {
+                const int v = sg * kSegVecs + lane;
+                float wv[PV];
+                float sum = v < nvec ? piece_vec_weights<T>(wr, nullptr, nullptr, 0, vec_ok, e0, n, v, wv) : 0.f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                if (lane == 0) s_tmp[sg] = sum;
+            }
+            __syncwarp();
+            segp = s_tmp;
+        }
+    }
+    if (pstar < 0) return -1;
+    return select_in_piece_body<T>(wr, segp, nullptr, nullptr, 0, vec_ok, pstar * p.PE,
+                                   min(p.V - pstar * p.PE, p.PE), local);
+}
+
 // ============================================================================
 // K2c: selection of the residual draws, one warp per queued residual draw.
 

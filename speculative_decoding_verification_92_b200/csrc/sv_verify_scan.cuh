@@ -167,15 +167,27 @@ __device__ __forceinline__ int warp_pick(const float (&w)[kMaxPer], int n, float
 constexpr int kMaxPieces = (SV_MAX_V * 4 + kPieceBytes - 1) / kPieceBytes;
 constexpr int kMaxPiecesPerLane = (kMaxPieces + 31) / 32;
 
-template <typename T>
-__global__ void __launch_bounds__(kScanThreads)
-verify_scan_kernel(const ScanParams p) {
-    extern __shared__ __align__(128) unsigned char scan_dsm[];
-    __shared__ int s_first, s_fail;
-    __shared__ float s_ustar;
+// The shared-memory scalars of one request's scan.
+struct ScanShared {
+    int first, fail;
+    float ustar;
+    DrawReq draw;
+};
 
+// Steps 1-5 for request b, by one CTA of kScanThreads threads (all of them
+// call it; scan_dsm holds scan_smem_bytes(k_max, P) bytes).  `outputs`: this
+// CTA writes the request's outputs (step 4); `queue`: the scan kernel's
+// form -- it lets the next grid launch before step 4 and queues the final
+// draw for the draw kernel itself.  Otherwise returns true when a final draw
+// follows (sampling, valid request), with the draw in ss->draw (visible to
+// every thread: the function ends with __syncthreads() then).
+template <typename T>
+__device__ __forceinline__ bool scan_request(const ScanParams& p, int b, unsigned char* scan_dsm, ScanShared* ss,
+                                             bool outputs, bool queue) {
+    int& s_first = ss->first;
+    int& s_fail = ss->fail;
+    float& s_ustar = ss->ustar;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.x;
     const int K = p.k_max;
     const int nslots = 2 * K + 1;  // partial rows per request
     const int P = p.P;
@@ -255,8 +267,8 @@ verify_scan_kernel(const ScanParams p) {
     // sums), and two shuffles combine the four.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (!ok) {
-        write_failed(-1);
-        return;
+        if (outputs) write_failed(-1);
+        return false;
     }
     if (tid == 0) { s_fail = 0; s_first = L; }
     const int n_t = L + 1;
@@ -322,8 +334,8 @@ verify_scan_kernel(const ScanParams p) {
     }
     __syncthreads();
     if (s_fail) {
-        write_failed(-2);
-        return;
+        if (outputs) write_failed(-2);
+        return false;
     }
 
     // 3. p, q at the drafted ids; acceptance scan ----------------------------------
@@ -371,23 +383,25 @@ verify_scan_kernel(const ScanParams p) {
                 p.out_expected_len[b] = e;
             }
         }
-        return;
+        return false;
     }
 
     // 4. outputs of the scan -----------------------------------------------------------
     // The draw kernel may be launched now (its CTAs then wait for this grid);
     // launching it earlier would let its waiting CTAs slow this grid down.
-    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
+    if (queue && tid == 0) asm volatile("griddepcontrol.launch_dependents;");
     const int j = s_first;
-    for (int i = tid; i <= K; i += kScanThreads) {
-        if (i < j) out_tok[i] = s_x[i];
-        else if (i > j) out_tok[i] = -1;
-        else if (p.greedy) out_tok[i] = s_arg_t[j];
+    if (outputs) {
+        for (int i = tid; i <= K; i += kScanThreads) {
+            if (i < j) out_tok[i] = s_x[i];
+            else if (i > j) out_tok[i] = -1;
+            else if (p.greedy) out_tok[i] = s_arg_t[j];
+        }
+        if (tid == 0) p.out_len[b] = j;
     }
-    if (tid == 0) p.out_len[b] = j;
-    if (p.greedy) return;
+    if (p.greedy) return false;
 
-    // 5. queue the final draw on row j ---------------------------------------------------
+    // 5. the final draw on row j ----------------------------------------------------------
     if (warp == 0) {
         DrawReq r;
         r.b = b;
@@ -426,7 +440,9 @@ verify_scan_kernel(const ScanParams p) {
             r.target = pc < 0 ? INFINITY : local;
         }
         if (lane == 0) {
-            if (r.mode == kResidual) {
+            if (!queue) {
+                ss->draw = r;
+            } else if (r.mode == kResidual) {
                 const int slot = atomicAdd(p.ctrl + 0, 1);
                 p.res_lost[slot] = 0;
                 p.res_req[slot] = r;
@@ -436,6 +452,17 @@ verify_scan_kernel(const ScanParams p) {
             }
         }
     }
+    if (queue) return false;
+    __syncthreads();
+    return true;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kScanThreads)
+verify_scan_kernel(const ScanParams p) {
+    extern __shared__ __align__(128) unsigned char scan_dsm[];
+    __shared__ ScanShared ss;
+    (void)scan_request<T>(p, blockIdx.x, scan_dsm, &ss, true, true);
 }
 
 }  // namespace sv

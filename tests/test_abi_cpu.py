@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 8, names
     for name in names:
         assert hasattr(lib, name), f"{name} is declared in include/ but not exported"
-    assert sv.abi_version() == 2
+    assert sv.abi_version() == 3
 
 
 def test_status_strings():
@@ -117,6 +117,10 @@ def test_bad_options():
     o = _Options()
     o.wait_timeout_us = -5
     assert call(opts=o) == Status.EINVAL
+    for path in (3, -1):                    # only AUTO, QUEUE and CLUSTER exist
+        o = _Options()
+        o.draw_path = path
+        assert call(opts=o) == Status.EINVAL
     for r in (-1, 5):                      # names no request of the B = 4 batch
         o = _Options()
         o.lost_copy_request = r
@@ -187,3 +191,12 @@ def test_size_limits_match_the_header():
     for dt in (sv.F32, sv.BF16):
         assert lib.spec_verify_workspace_bytes(ctypes.byref(_Shape(3, sv.MAX_K, sv.MAX_V, dt, 0))) > 0
         assert lib.spec_verify_workspace_bytes(ctypes.byref(_Shape(3, 2, sv.MAX_V + 1, dt, 0))) == 0
+
+
+def test_auto_draw_path_rejects_bad_shapes_and_needs_a_gpu():
+    lib = sv.library()
+    assert lib.spec_verify_auto_draw_path(ctypes.byref(_Shape(4, 4, 0, sv.F32, 0))) == -1
+    assert lib.spec_verify_auto_draw_path(ctypes.byref(_Shape(-1, 4, 10, sv.F32, 0))) == -1
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.spec_verify_auto_draw_path(ctypes.byref(_Shape(4, 4, 1000, sv.F32, 0))) == -1

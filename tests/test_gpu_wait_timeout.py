@@ -64,12 +64,13 @@ def draw_victims(clean_len, w):
     return resid[:1] + bonus[:1]
 
 
+@pytest.mark.parametrize("path", [sv.DrawPath.QUEUE, sv.DrawPath.CLUSTER])
 @pytest.mark.parametrize("V,dtype,mode,misalign", [(1000, F32, "logits", False), (151936, BF16, "logits", False),
                                                    (151936, BF16, "ids", False), (4099, F32, "logits", True)])
-def test_lost_draw_copy_times_out_and_the_context_stays_usable(V, dtype, mode, misalign):
-    """The draw kernel's waits on its own bulk copies are bounded too:
-    ``lost_draw_request`` makes it skip the first staging of one request's
-    draw, that wait runs out, and the request reports -2."""
+def test_lost_draw_copy_times_out_and_the_context_stays_usable(V, dtype, mode, misalign, path):
+    """The draw's waits on its own bulk copies are bounded too, on both
+    draw paths: ``lost_draw_request`` makes the draw skip the first staging
+    of one request's draw, that wait runs out, and the request reports -2."""
     w = make_workload(B=12, k_max=4, V=V, dtype=dtype, seed=73, boost=3.0, draft_noise=0.5, draft_mode=mode,
                       lens=[4, 3, 4, 2, 4, 4, 1, 4, 0, 4, 3, 4])
     d = device_inputs(w, misalign=misalign)
@@ -77,7 +78,7 @@ def test_lost_draw_copy_times_out_and_the_context_stays_usable(V, dtype, mode, m
 
     def run(**kw):
         n, t = sv.spec_verify(d["target"], d["draft"], d["tokens"], d["lens"], d["uniforms"], w.temperature,
-                              V=w.V, stats_kernel=kernel, **kw)
+                              V=w.V, stats_kernel=kernel, draw_path=path, **kw)
         torch.cuda.synchronize()
         return n.cpu().numpy(), t.cpu().numpy()
 
