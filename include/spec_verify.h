@@ -155,7 +155,7 @@ typedef struct {
 typedef enum {
     SV_DRAW_AUTO = 0,
     SV_DRAW_QUEUE = 1,    /* scan kernel, draw kernel, selection kernel */
-    SV_DRAW_CLUSTER = 2   /* one cluster of up to 8 CTAs per request */
+    SV_DRAW_CLUSTER = 2   /* one cluster of up to 16 CTAs per request */
 } sv_draw_path;
 
 /* Bytes of device workspace spec_verify / spec_verify_stats need for this

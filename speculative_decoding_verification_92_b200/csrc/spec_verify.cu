@@ -310,15 +310,62 @@ cudaError_t launch_stats(const StatsParams& base, int B, int variant, const Devi
 // K2a (one CTA per request), then for sampling K2b (persistent, one wave) and,
 // with draft logits, K2c (one warp per possible residual draw), each a
 // programmatic dependent of the kernel before it.
+// Largest cluster size the cluster kernel uses with `smem` bytes of dynamic
+// shared memory: 16 when the device can place at least one such cluster
+// (non-portable size, opted into here), else the portable 8.  Cached per
+// context and size.
+std::map<std::pair<unsigned long long, size_t>, int> g_cluster_max;
+
+template <typename T>
+cudaError_t cluster_max_ctas(size_t smem, int* cmax) {
+    auto k = verify_cluster_kernel<T>;
+    const auto key = std::make_pair(current_context_id(), smem);
+    if (key.first != 0) {
+        std::lock_guard<std::mutex> lock(g_setup_mutex);
+        const auto it = g_cluster_max.find(key);
+        if (it != g_cluster_max.end()) {
+            *cmax = it->second;
+            return cudaSuccess;
+        }
+    }
+    // the kernel's shared-memory attributes first: the query below uses them
+    if (const cudaError_t e = kernel_setup(k, smem, kScanThreads, nullptr); e != cudaSuccess) return e;
+    int result = kClusterPortableCtas;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kClusterMaxCtas;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kClusterMaxCtas);
+        cfg.blockDim = dim3(kScanThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) == cudaSuccess && n > 0) result = kClusterMaxCtas;
+    }
+    (void)cudaGetLastError();  // a refused query leaves no error behind
+    if (key.first != 0) {
+        std::lock_guard<std::mutex> lock(g_setup_mutex);
+        g_cluster_max[key] = result;
+    }
+    *cmax = result;
+    return cudaSuccess;
+}
+
 // AUTO's choice: the cluster path when the batch's CTAs fit in half of one
 // resident wave of the cluster kernel (clusters are placed whole, inside one
 // GPC), so every request's cluster starts at once.
 template <typename T>
 cudaError_t cluster_fits(int B, int k_max, int P, const DeviceInfo& dev, bool* fits) {
-    int per_sm = 0;
-    const cudaError_t e = kernel_setup(verify_cluster_kernel<T>, cluster_smem_bytes(k_max, P), kScanThreads, &per_sm);
+    int per_sm = 0, cmax = 0;
+    const size_t smem = cluster_smem_bytes(k_max, P);
+    cudaError_t e = kernel_setup(verify_cluster_kernel<T>, smem, kScanThreads, &per_sm);
+    if (e == cudaSuccess) e = cluster_max_ctas<T>(smem, &cmax);
     if (e != cudaSuccess) return e;
-    *fits = int64_t(B) * cluster_ctas(P) * 2 <= int64_t(per_sm) * dev.sm_count;
+    *fits = int64_t(B) * cluster_ctas(P, cmax) * 2 <= int64_t(per_sm) * dev.sm_count;
     return cudaSuccess;
 }
 
@@ -332,8 +379,10 @@ cudaError_t launch_cluster(const ScanParams& sp, const DrawParams& dp, int B, in
     *launched = false;
     if (path == SV_DRAW_QUEUE) return cudaSuccess;
     auto k = verify_cluster_kernel<T>;
-    const int C = cluster_ctas(dp.P);
     const size_t smem = cluster_smem_bytes(dp.k_max, dp.P);
+    int cmax = 0;
+    if (const cudaError_t e = cluster_max_ctas<T>(smem, &cmax); e != cudaSuccess) return e;
+    const int C = cluster_ctas(dp.P, cmax);
     if (path == SV_DRAW_AUTO) {
         bool fits = false;
         const cudaError_t e = cluster_fits<T>(B, dp.k_max, dp.P, dev, &fits);

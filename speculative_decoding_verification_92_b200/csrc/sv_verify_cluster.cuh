@@ -30,13 +30,15 @@
 
 namespace sv {
 
-constexpr int kClusterMaxCtas = 8;  // portable cluster size
-// pieces per CTA: C = P below 8 pieces (one each), else C = 8
-constexpr int kClusterMaxPerCta = (kMaxPieces + kClusterMaxCtas - 1) / kClusterMaxCtas;
+// CTAs per cluster: min(P, cmax) with cmax = 16 (a non-portable cluster
+// size, used where the GPU can place such clusters) or else 8 (portable).
+constexpr int kClusterMaxCtas = 16;
+constexpr int kClusterPortableCtas = 8;
+// pieces per CTA: at most ceil(P / 8)
+constexpr int kClusterMaxPerCta = (kMaxPieces + kClusterPortableCtas - 1) / kClusterPortableCtas;
 constexpr size_t kClusterBufBytes = kDrawBufBytes;        // one staging buffer: a target and a draft piece
 
-// CTAs per cluster for a row of P pieces.
-__host__ __device__ inline int cluster_ctas(int P) { return P < kClusterMaxCtas ? (P < 1 ? 1 : P) : kClusterMaxCtas; }
+__host__ __device__ inline int cluster_ctas(int P, int cmax) { return P < cmax ? (P < 1 ? 1 : P) : cmax; }
 
 // Dynamic shared memory of the cluster kernel: the scan's area, then two
 // staging buffers.

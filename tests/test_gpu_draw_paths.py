@@ -57,7 +57,7 @@ def test_misaligned_rows_on_both_paths():
 
 
 def test_largest_vocabulary_on_both_paths():
-    # P = 96 fp32 pieces: 12 per CTA of the cluster, more than 32 per selection warp lane row
+    # P = 96 fp32 pieces: several per CTA of the cluster, more than 32 per selection warp
     w = make_workload(B=3, k_max=2, V=sv.MAX_V, dtype=F32, seed=84, z_sigma=4.0, boost=0.0, draft_noise=0.5,
                       lens=[2, 1, 2])
     both_paths(w)
