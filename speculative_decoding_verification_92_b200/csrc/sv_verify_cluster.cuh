@@ -211,7 +211,15 @@ verify_cluster_kernel(const ScanParams sp, const DrawParams p) {
                     __syncwarp();
                     return s_sel;
                 };
-                const int tok = select_residual_warp<T>(p, r, w, seg_of, s_sel);
+                // a CTA with at most two pieces still holds both in its buffers
+                // (piece k in buffer k): the selection reads the chosen one there
+                auto stage_of = [&](int c) -> StagedPiece {
+                    const int owner = c % C, k = c / C;
+                    if ((P - 1 - owner) / C + 1 > 2) return StagedPiece{nullptr, nullptr, 0};
+                    const unsigned char* tb = cluster.map_shared_rank(bufs + size_t(k) * kClusterBufBytes, owner);
+                    return StagedPiece{tb, tb + kPieceBytes, staged_bytes(c) / 16};
+                };
+                const int tok = select_residual_warp<T>(p, r, w, seg_of, stage_of, s_sel);
                 if (tok >= 0) {
                     if (lane == 0) out[r.j] = tok;
                 } else {

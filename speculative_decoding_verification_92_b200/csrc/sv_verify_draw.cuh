@@ -100,12 +100,15 @@ struct WeightRow {
 // Up to PV logits of one row starting at element idx0 (count < PV: the rest
 // are -inf), from shared memory when `sm` is given, else from global memory
 // (16-byte load when `vec_ok` and the vector is whole).
-template <typename T>
+// kGeneric: `sm` is a generic address (another CTA's shared memory in the
+// cluster) rather than this CTA's.
+template <typename T, bool kGeneric = false>
 __device__ __forceinline__ void load_vec(const unsigned char* sm, const unsigned char* row, int idx0, int count,
                                          bool vec_ok, float (&z)[Logit<T>::kPerVec]) {
     constexpr int PV = Logit<T>::kPerVec;
     if (sm) {
-        Logit<T>::unpack(ld_shared_v4(sm), z);
+        if constexpr (kGeneric) Logit<T>::unpack(*reinterpret_cast<const uint4*>(sm), z);
+        else Logit<T>::unpack(ld_shared_v4(sm), z);
     } else if (vec_ok && count == PV) {
         Logit<T>::unpack(ld_global_stream_v4(row + int64_t(idx0) * Logit<T>::kSize), z);
     } else {
@@ -138,7 +141,7 @@ __device__ __forceinline__ float vec_weights(const WeightRow& r, const float (&z
 
 // Weights of vector v of piece pc (elements [e0, e0 + n) of the row), from
 // the staged copy when it holds the vector, else from global memory.
-template <typename T>
+template <typename T, bool kGeneric = false>
 __device__ __forceinline__ float piece_vec_weights(const WeightRow& r, const unsigned char* tbuf,
                                                    const unsigned char* dbuf, int nstaged_vec, bool vec_ok, int e0,
                                                    int n, int v, float (&w)[Logit<T>::kPerVec]) {
@@ -147,8 +150,8 @@ __device__ __forceinline__ float piece_vec_weights(const WeightRow& r, const uns
     const int count = min(PV, n - v * PV);
     float z[PV], y[PV];
     const bool staged = v < nstaged_vec;
-    load_vec<T>(staged ? tbuf + 16 * v : nullptr, r.trow, idx0, count, vec_ok, z);
-    if (r.mode == kResidual) load_vec<T>(staged ? dbuf + 16 * v : nullptr, r.drow, idx0, count, vec_ok, y);
+    load_vec<T, kGeneric>(staged ? tbuf + 16 * v : nullptr, r.trow, idx0, count, vec_ok, z);
+    if (r.mode == kResidual) load_vec<T, kGeneric>(staged ? dbuf + 16 * v : nullptr, r.drow, idx0, count, vec_ok, y);
 #pragma unroll
     for (int i = 0; i < PV; ++i)
         if (r.mode != kResidual) y[i] = 0.f;
@@ -251,7 +254,7 @@ __device__ __forceinline__ void piece_segments(const WeightRow& r, const unsigne
 // `target` -- segment (scan over lanes), vector (one vector per lane, a scan
 // over lanes) and element.  Returns the row index (same in every lane), or -1
 // when the piece has no positive weight.
-template <typename T>
+template <typename T, bool kGeneric = false>
 __device__ __forceinline__ int select_in_piece_body(const WeightRow& r, const float* seg, const unsigned char* tbuf,
                                                     const unsigned char* dbuf, int nstaged_vec, bool vec_ok, int e0,
                                                     int n, float target) {
@@ -267,7 +270,7 @@ __device__ __forceinline__ int select_in_piece_body(const WeightRow& r, const fl
     float sum = 0.f;
 #pragma unroll
     for (int i = 0; i < PV; ++i) w[i] = 0.f;
-    if (v < nvec) sum = piece_vec_weights<T>(r, tbuf, dbuf, nstaged_vec, vec_ok, e0, n, v, w);
+    if (v < nvec) sum = piece_vec_weights<T, kGeneric>(r, tbuf, dbuf, nstaged_vec, vec_ok, e0, n, v, w);
     const float lv = warp_scan_incl(sum);
     const unsigned cross = __ballot_sync(0xffffffffu, sum > 0.f && lv > t_seg);
     const unsigned pos = __ballot_sync(0xffffffffu, sum > 0.f);
@@ -647,21 +650,30 @@ verify_draw_kernel(const DrawParams p) {
     }
 }
 
+// A staged copy of a residual piece: target and draft bytes (generic
+// addresses) and the 16-byte vectors they hold; tbuf == nullptr: none.
+struct StagedPiece {
+    const unsigned char* tbuf;
+    const unsigned char* dbuf;
+    int nvec;
+};
+
 // One warp: the residual draw r from its piece totals w (lane l holding
 // pieces [l*cps, l*cps + cps)): the piece and the segment holding u*W, then
 // the vector and the element, re-reading that segment of both rows
 // (seg_of(c) returns piece c's 32 segment sums where the whole warp can read
-// them).  Zero residual mass (p == q numerically) draws from p_j instead:
+// them; stage_of(c) the piece's staged copy when one is still held, whose
+// vectors are then read instead of global memory).  Zero residual mass (p == q numerically) draws from p_j instead:
 // the piece from the partials, its segment sums computed here by the warp
 // into s_tmp (32 floats).  Returns the token, or -1 when no positive weight
 // is found (not reached with finite logits).  Used by the cluster kernel;
 // the selection kernel below takes the same steps inline, interleaved with
 // its loads (0.7 us per step faster on the largest workload than calling
 // this function).  Their picks are identical.
-template <typename T, typename Params, typename SegOf>
+template <typename T, typename Params, typename SegOf, typename StageOf>
 __device__ __forceinline__ int select_residual_warp(const Params& p, const DrawReq& r,
                                                     const float (&w)[kMaxPiecesPerLane], SegOf seg_of,
-                                                    float* s_tmp) {
+                                                    StageOf stage_of, float* s_tmp) {
     constexpr int PV = Logit<T>::kPerVec;
     const int lane = threadIdx.x & 31;
     const int K = p.k_max;
@@ -723,6 +735,13 @@ __device__ __forceinline__ int select_residual_warp(const Params& p, const DrawR
         }
     }
     if (pstar < 0) return -1;
+    if (wr.mode == kResidual) {
+        // the piece's staged copy, where it is still held (a generic address)
+        const StagedPiece sp = stage_of(pstar);
+        if (sp.tbuf)
+            return select_in_piece_body<T, true>(wr, segp, sp.tbuf, sp.dbuf, sp.nvec, vec_ok, pstar * p.PE,
+                                                 min(p.V - pstar * p.PE, p.PE), local);
+    }
     return select_in_piece_body<T>(wr, segp, nullptr, nullptr, 0, vec_ok, pstar * p.PE,
                                    min(p.V - pstar * p.PE, p.PE), local);
 }
