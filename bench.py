@@ -81,6 +81,8 @@ def parse_args():
     ap.add_argument("--config", type=int, default=5, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--stats-kernel", default="auto", choices=["auto", "tma", "vec16", "scalar"])
+    ap.add_argument("--draw-path", default="auto", choices=["auto", "queue", "cluster"],
+                    help="how sampling calls make their final draws (the library's AUTO by default)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -518,9 +520,9 @@ class DeviceWorkload:
     logits from HBM, as a fresh batch would be, and no cache flush (whose
     dirty lines would be written back inside the timed step) is needed."""
 
-    def __init__(self, sv, torch, dev, stream, w, greedy, kernel):
+    def __init__(self, sv, torch, dev, stream, w, greedy, kernel, draw_path=0):
         self.sv, self.torch, self.dev, self.stream, self.w = sv, torch, dev, stream, w
-        self.greedy, self.kernel = greedy, kernel
+        self.greedy, self.kernel, self.draw_path = greedy, kernel, draw_path
         self.is_bf16 = w.dtype == "bf16"
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         self.in_bytes = input_bytes(w, greedy)
@@ -560,7 +562,7 @@ class DeviceWorkload:
         pick = lambda x: None if x is None else x[c]
         self.sv.spec_verify(pick(self.target), pick(self.draft), pick(self.tokens), pick(self.lens),
                             pick(self.uniforms), w.temperature, self.greedy, V=w.V, out=self.out, workspace=self.ws,
-                            stream=self.stream, stats_kernel=self.kernel, events=events)
+                            stream=self.stream, stats_kernel=self.kernel, events=events, draw_path=self.draw_path)
 
     def event(self):
         e = self.torch.cuda.Event(enable_timing=True)
@@ -655,11 +657,14 @@ def reread_bytes(w, g_len, greedy=False) -> int:
     return int((1 + resid.astype(np.int64)).sum()) * w.V * w.esize
 
 
-def draw_path_of(sv, w, greedy) -> str:
-    """The draw path the library's AUTO choice takes for this workload
-    ("cluster" or "queue"; greedy calls make no draw)."""
+def draw_path_of(sv, w, greedy, forced=0) -> str:
+    """The draw path a call takes for this workload: `forced` (a DrawPath)
+    or else the library's AUTO choice ("cluster" or "queue"; greedy calls
+    make no draw)."""
     if greedy:
         return "none"
+    if forced:
+        return "cluster" if forced == sv.DrawPath.CLUSTER else "queue"
     dt = sv.BF16 if w.dtype == "bf16" else sv.F32
     path = sv.auto_draw_path(w.B, w.k_max, w.V, dt, w.target.shape[2])
     return "cluster" if path == sv.DrawPath.CLUSTER else "queue"
@@ -698,7 +703,7 @@ def config_record(dw, cfg, steps, warmup, k1_samples, peak):
         "k1_gbs_median": alg / (k1_med / 1e3) / 1e9, "k1_frac_median": alg / (k1_med / 1e3) / 1e9 / peak,
         "k1_frac_mean": alg / (k1_mean / 1e3) / 1e9 / peak,
         "accept_rate": float(g_len.sum() / max(1, w.positions)), "mean_accept_len": float(g_len.mean()),
-        "draw_path": draw_path_of(dw.sv, w, dw.greedy), "parity": parity,
+        "draw_path": draw_path_of(dw.sv, w, dw.greedy, dw.draw_path), "parity": parity,
     }
 
 
@@ -730,7 +735,8 @@ def run_ours_impl(args):
     stream = torch.cuda.current_stream()
     peak, peak_kind = measured_peak()
     w = make_rank_workload(args.config, rank)
-    dw = DeviceWorkload(sv, torch, dev, stream, w, greedy, kernel)
+    draw_path = {"auto": sv.DrawPath.AUTO, "queue": sv.DrawPath.QUEUE, "cluster": sv.DrawPath.CLUSTER}[args.draw_path]
+    dw = DeviceWorkload(sv, torch, dev, stream, w, greedy, kernel, draw_path)
 
     K, W = args.steps, args.warmup
     with ClockSampler(local_rank) as clocks:
@@ -804,7 +810,7 @@ def run_ours_impl(args):
     cfgd.update({"parallelism": f"replicas{n}" if n > 1 else "single",
                  "sharding": "each rank verifies its own batch; no data-path collective",
                  "l2": dw.l2_note, "stats_kernel": variant, "greedy": greedy,
-                 "draw_path": draw_path_of(sv, w, greedy)})
+                 "draw_path": draw_path_of(sv, w, greedy, draw_path)})
     dw.release()
 
     # ---------------- the other workloads (rank 0, N = 1) ----------------
@@ -815,7 +821,7 @@ def run_ours_impl(args):
             if cfg == args.config:
                 continue
             wc = make_rank_workload(cfg, 0)
-            dc = DeviceWorkload(sv, torch, dev, stream, wc, greedy, kernel)
+            dc = DeviceWorkload(sv, torch, dev, stream, wc, greedy, kernel, draw_path)
             per_config[str(cfg)] = config_record(dc, cfg, args.per_config_steps, max(W, 3),
                                                  max(args.k1_samples, 10), peak)
             dc.release()
@@ -832,7 +838,7 @@ def run_ours_impl(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": K, "warmup": W,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic", "config": cfgd,
-            "e2e": e2e, "gpu_launches": K * launches_per_call(w.B, draw_path_of(sv, w, greedy), w.draft is not None), "roofline": roofline,
+            "e2e": e2e, "gpu_launches": K * launches_per_call(w.B, draw_path_of(sv, w, greedy, draw_path), w.draft is not None), "roofline": roofline,
             "cpu_baseline": cpu, "clocks": clocks.summary(),
             "hbm_gbs": alg / (ms_per_step / 1e3) / 1e9,
             "accept_rate": accept_rate, "mean_accept_len": float(g_len.mean()),
