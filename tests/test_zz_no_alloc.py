@@ -46,8 +46,9 @@ def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
     w1 = make_config(2)                                   # 64 x 17 rows x 19 pieces of partials
     w2 = make_workload(B=33, k_max=12, V=20000, dtype="f32", seed=5, boost=4.0, draft_noise=0.3,
                        lens_choices=(0, 4, 12), lens_probs=(0.4, 0.3, 0.3))
+    w3 = make_config(4)                                   # a small batch: the cluster draw path
     assert sv.workspace_bytes(w1.B, w1.k_max, w1.V, sv.BF16) <= SCRATCH_BYTES
-    for w in (w1, w2, w1):
+    for w in (w1, w2, w3, w1):
         d = device_inputs(w)
         want_len, want_tok = run_gpu(w, inputs=d)
         st, got_len, got_tok = call_static(w, d)
