@@ -14,8 +14,10 @@
 //      keeps each piece's 32 segment sums and total in its shared memory;
 //      after a cluster barrier CTA 0 reads every piece total through
 //      distributed shared memory, picks the piece and the segment holding
-//      u*W, re-reads that segment of both rows and picks the vector and the
-//      element (select_residual_warp, shared with the selection kernel);
+//      u*W, reads that segment of both rows (from the staging buffer of the
+//      CTA that holds the piece when it still holds it, else from global
+//      memory) and picks the vector and the element (select_residual_warp:
+//      the selection kernel's steps);
 //   3. bonus and one-hot draws: CTA 0 alone, as one task of the draw kernel.
 // The weights, the selection order and the fallbacks are the draw kernel's
 // ("AI 开始抄自己的作业——而且抄得理直气壮", section "⚡ 投机解码：让草稿先跑，考官殿后").
