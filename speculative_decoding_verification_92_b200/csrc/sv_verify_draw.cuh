@@ -439,9 +439,10 @@ verify_draw_kernel(const DrawParams p) {
         }
         mbar_arrive_expect_tx(&s_bar[buf], resid ? 2 * nb : nb);
         const int64_t off = int64_t(pc) * p.PE * esz;
-        const uint64_t pol = l2_evict_first_policy();  // each piece is staged once
-        bulk_copy_g2s_hint(dst, trow_of(r) + off, nb, &s_bar[buf], pol);
-        if (resid) bulk_copy_g2s_hint(dst + kPieceBytes, drow_of(r) + off, nb, &s_bar[buf], pol);
+        // default L2 policy: the selection kernel re-reads one segment of the
+        // chosen piece right after this kernel, and finds it in L2
+        bulk_copy_g2s(dst, trow_of(r) + off, nb, &s_bar[buf]);
+        if (resid) bulk_copy_g2s(dst + kPieceBytes, drow_of(r) + off, nb, &s_bar[buf]);
     };
     // All threads: wait for buffer buf's pending completion (bounded);
     // block-uniform result.  On success the parity moves on; on a timeout it
